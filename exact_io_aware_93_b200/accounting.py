@@ -1,0 +1,36 @@
+"""Work and traffic accounting used by the benchmark (no attention arithmetic).
+
+FLOP convention: the forward pass does two B*H*N*N*d contractions (Q K^T and
+P V) at 2 flop per multiply-add, i.e. 4*B*H*N^2*d, halved when causal; the
+backward pass counts 2.5x the forward.
+
+Algorithmic bytes are the bytes a kernel must move at minimum: each operand
+read once, each result written once (bf16 tensors 2 bytes per element, fp32
+statistics 4 bytes).
+"""
+from __future__ import annotations
+
+
+def fwd_flops(B: int, H: int, N: int, d: int, causal: bool) -> float:
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def bwd_flops(B: int, H: int, N: int, d: int, causal: bool) -> float:
+    return 2.5 * fwd_flops(B, H, N, d, causal)
+
+
+def fwd_bytes(B: int, H: int, N: int, d: int) -> int:
+    """Q, K, V read and O written (bf16), LSE written (fp32)."""
+    return 2 * 4 * B * H * N * d + 4 * B * H * N
+
+
+def bwd_bytes(B: int, H: int, N: int, d: int) -> int:
+    """Q, K, V, O, dO read and dQ, dK, dV written (bf16); LSE and D (fp32) read/written once;
+    the fp32 dQ accumulator written once and read once."""
+    return 2 * 8 * B * H * N * d + 3 * 4 * B * H * N + 2 * 4 * B * H * N * d
+
+
+def score_matrix_bytes(N: int, heads: int, bytes_per_score: int = 2) -> int:
+    """Size of the N x N score matrix standard attention would materialise."""
+    return N * N * heads * bytes_per_score

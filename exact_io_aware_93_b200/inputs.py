@@ -1,0 +1,119 @@
+"""Seeded synthetic workloads shared by the tests, the benchmark and the smoke check.
+
+This module only draws random numbers and picks rows; it holds none of the
+attention arithmetic, and neither the CUDA path nor the oracle depends on it.
+
+Recipe (the same for every workload):
+
+* ``torch.Generator('cpu')`` seeded with the workload's seed draws fp32
+  standard normals in the order Q, K, V, dO, each of shape
+  ``[B, N, H, d]`` (batch, sequence, heads, head_dim -- the layout of the
+  ``flash_attn_func`` interface in the holysheep.ai review, section
+  "Implementing Flash Attention in Your Architecture").
+* For the peaked workload, a seeded permutation picks floor(N/100) sequence
+  positions (shared by all batches and heads) and the whole K vector at those
+  positions is multiplied by 3 in fp32, before rounding.
+* Every tensor is then rounded to bfloat16 (round to nearest even); the same
+  bf16 values are handed to the GPU and, widened exactly to fp64, to the
+  oracle.
+* Checked query rows: per (b, h) a seeded sample without replacement from
+  [0, N), always including rows 0, 1 and N-1.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    seed: int
+    backward: bool = False
+    peaked: bool = False
+    # forward rows checked per head (None = every row)
+    rows_per_head: int | None = None
+    # backward: heads checked in full, plus (extra_heads x extra_rows_per_head) sampled rows
+    bwd_full_heads: int = 0
+    bwd_extra_heads: int = 0
+    bwd_extra_rows: int = 0
+    notes: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(self.d) ** 0.5
+
+
+# The five workloads: shapes, seeds and checked-row counts.
+WORKLOADS = {
+    w.name: w
+    for w in [
+        Workload("tiny_b1_h1_n256_d64", 1, 1, 256, 64, False, 1001,
+                 notes="tiny non-causal forward, every row checked"),
+        Workload("causal_b4_h16_n2048_d128", 4, 16, 2048, 128, True, 1002,
+                 rows_per_head=None,
+                 notes="causal forward, every row of every head checked"),
+        Workload("causal_b1_h32_n32768_d128", 1, 32, 32768, 128, True, 1003,
+                 rows_per_head=4096,
+                 notes="long-context causal forward, 4096 rows per head"),
+        Workload("causal_fwdbwd_b2_h16_n8192_d128", 2, 16, 8192, 128, True, 1004,
+                 backward=True, bwd_full_heads=2, bwd_extra_heads=4, bwd_extra_rows=256,
+                 notes="causal forward + recompute backward; 2 full heads + 1024 rows elsewhere"),
+        Workload("causal_peaked_b1_h8_n131072_d128", 1, 8, 131072, 128, True, 1005,
+                 peaked=True, rows_per_head=512,
+                 notes="very long causal forward, K x3 on 1% of positions, 512 rows per head"),
+    ]
+}
+
+
+def peaked_positions(N: int, gen: torch.Generator) -> torch.Tensor:
+    """floor(N/100) distinct sequence positions, drawn by a seeded permutation."""
+    return torch.randperm(N, generator=gen)[: N // 100]
+
+
+def make_inputs(B: int, H: int, N: int, d: int, seed: int, *, with_do: bool = False,
+                peaked: bool = False) -> dict[str, torch.Tensor]:
+    """CPU bf16 tensors ``q, k, v`` (and ``do``) of shape [B, N, H, d]."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    shape = (B, N, H, d)
+    out = {}
+    names = ["q", "k", "v"] + (["do"] if with_do else [])
+    for name in names:
+        out[name] = torch.randn(shape, generator=gen, dtype=torch.float32)
+    if peaked:
+        pos = peaked_positions(N, gen)
+        out["k"][:, pos] *= 3.0
+        out["peaked_positions"] = pos
+    for name in names:
+        out[name] = out[name].to(torch.bfloat16)
+    return out
+
+
+def make_workload_inputs(w: Workload) -> dict[str, torch.Tensor]:
+    return make_inputs(w.B, w.H, w.N, w.d, w.seed, with_do=w.backward, peaked=w.peaked)
+
+
+def sample_rows(N: int, count: int | None, seed: int) -> torch.Tensor:
+    """Sorted distinct rows in [0, N): a seeded sample of ``count`` plus {0, 1, N-1}.
+
+    ``count=None`` (or count >= N) returns every row.
+    """
+    if count is None or count >= N:
+        return torch.arange(N, dtype=torch.int64)
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    picked = torch.randperm(N, generator=gen)[:count]
+    fixed = torch.tensor([0, min(1, N - 1), N - 1], dtype=torch.int64)
+    return torch.unique(torch.cat([picked, fixed]))
+
+
+def head_row_seed(w_seed: int, b: int, h: int) -> int:
+    """Per-(batch, head) seed for row sampling."""
+    return int(w_seed) * 1_000_003 + b * 1009 + h * 7 + 17
