@@ -1,0 +1,125 @@
+"""Thin Python binding of the C ABI in ``include/fa.h`` (argument marshalling only).
+
+Every step of the computation runs in ``libfa_b200.so``; this module checks
+tensor shapes the way the ``validate_attention_inputs`` helper of the
+holysheep.ai review does (section "Common Errors and Fixes", error 4: same
+batch, heads and head_dim for Q, K, V; same sequence length for K and V),
+allocates outputs with PyTorch and passes raw device pointers.  There is no
+fallback: without the compiled library, a CUDA tensor or an sm_100 device the
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+from . import build as _build
+
+_lib = None
+
+FA_STATUS = {
+    0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_ALIGNMENT",
+    4: "FA_ERR_DEVICE", 5: "FA_ERR_LAUNCH", 6: "FA_ERR_TIMEOUT", 7: "FA_ERR_WORKSPACE",
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = int(status)
+        super().__init__(f"{what}: {FA_STATUS.get(int(status), 'FA_ERR_UNKNOWN')} ({int(status)})")
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libfa_b200.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise FileNotFoundError(
+            f"{path} is missing; build it with `python -m exact_io_aware_93_b200.build` "
+            "(there is no non-CUDA fallback)")
+    L = ctypes.CDLL(path)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    L.fa_abi_version.restype = i
+    L.fa_status_string.argtypes = [i]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    L.fa_fwd.restype = i
+    L.fa_get_status.argtypes = [vp]
+    L.fa_get_status.restype = i
+    if hasattr(L, "fa_bwd"):
+        L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+        L.fa_bwd_workspace_size.restype = ctypes.c_size_t
+        L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                             i, i, i, i, f, i, vp]
+        L.fa_bwd.restype = i
+    _lib = L
+    return L
+
+
+def _stream_ptr(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def validate_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [batch, seq_len, num_heads, head_dim], got {tuple(t.shape)}")
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.shape[0] == k.shape[0] == v.shape[0]):
+        raise ValueError(f"batch size mismatch: {q.shape[0]}, {k.shape[0]}, {v.shape[0]}")
+    if not (q.shape[2] == k.shape[2] == v.shape[2]):
+        raise ValueError(f"num heads mismatch: {q.shape[2]}, {k.shape[2]}, {v.shape[2]}")
+    if k.shape[1] != v.shape[1]:
+        raise ValueError(f"key/value sequence length mismatch: {k.shape[1]}, {v.shape[1]}")
+    if not (q.shape[3] == k.shape[3] == v.shape[3]):
+        raise ValueError(f"head dim mismatch: {q.shape[3]}, {k.shape[3]}, {v.shape[3]}")
+    if q.shape[1] != k.shape[1]:
+        raise ValueError(f"query and key sequence lengths must match: {q.shape[1]}, {k.shape[1]}")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on the same device")
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+        scale: float | None = None, out: torch.Tensor | None = None,
+        lse: torch.Tensor | None = None):
+    """(O [B, N, H, d] bf16, LSE [B, H, N] fp32) of exact attention via ``fa_fwd``."""
+    validate_inputs(q, k, v)
+    B, N, H, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                      B, H, N, d, ctypes.c_float(scale), int(bool(causal)), _stream_ptr(q))
+    if st != 0:
+        raise FAError(st, "fa_fwd")
+    return out, lse
+
+
+def get_status(device: torch.device | None = None) -> int:
+    """Synchronise the current stream and read-and-clear the device status word."""
+    s = torch.cuda.current_stream(device)
+    return int(lib().fa_get_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None) -> torch.Tensor:
+    """O only."""
+    return fwd(q, k, v, causal=causal, scale=scale)[0]

@@ -1,0 +1,153 @@
+// fa_api.cu -- the C ABI of include/fa.h: argument validation, TMA tensor maps,
+// per-device kernel setup and launches of the sm_100a kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/fa.h"
+#include "fa_fwd_kernel.cuh"
+#include "tma_host.h"
+
+// Device status word: [0] = first error code a kernel recorded, [1] = wait site.
+__device__ int g_fa_status[2];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool ok = false;
+  int sm_count = 0;
+  int* status = nullptr;
+  bool fwd_attr[2][2] = {{false, false}, {false, false}};  // [d==128][causal]
+};
+DeviceInfo g_dev[kMaxDevices];
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+fa_status current_device(DeviceInfo** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_DEVICE;
+  }
+  DeviceInfo& di = g_dev[dev];
+  if (!di.probed) {
+    di.probed = true;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_DEVICE;
+    }
+    void* sym = nullptr;
+    if (prop.major == 10 && prop.minor == 0 && cudaGetSymbolAddress(&sym, g_fa_status) == cudaSuccess) {
+      di.ok = true;
+      di.sm_count = prop.multiProcessorCount;
+      di.status = static_cast<int*>(sym);
+    }
+    cudaGetLastError();
+  }
+  if (!di.ok) return FA_ERR_DEVICE;
+  *out = &di;
+  return FA_OK;
+}
+
+fa_status check_common(int B, int H, int N, int d, float scale, int causal) {
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  // every element index and every tile count must stay in range
+  const long double elems = static_cast<long double>(B) * N * H * d;
+  if (elems > static_cast<long double>(INT64_MAX / 4)) return FA_ERR_INVALID_ARG;
+  const long long nkb = (static_cast<long long>(N) + 127) / 128;
+  if (static_cast<long long>(B) * H * ((nkb + 1) / 2) > INT32_MAX) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o,
+                     float* lse, int B, int H, int N, float scale, cudaStream_t stream) {
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
+  const int smem = static_cast<int>(sizeof(fa::FwdSmem<D>)) + 1024;
+  bool& attr = di.fwd_attr[D == 128][CAUSAL];
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    attr = true;
+  }
+  const long long nkb = (static_cast<long long>(N) + 127) / 128;
+  const long long tiles = static_cast<long long>(B) * H * ((nkb + 1) / 2);
+  const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
+  const float scale_log2 = scale * 1.4426950408889634f;
+  kern<<<grid, fa::kFwdThreads, smem, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, B, H, N,
+                                                 scale_log2, di.status);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_abi_version(void) { return 1; }
+
+const char* fa_status_string(int s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT";
+    case FA_ERR_DEVICE: return "FA_ERR_DEVICE";
+    case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  st = current_device(&di);
+  if (st != FA_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if (!fa::make_bshd_map(&mq, q, B, N, H, d, 128) || !fa::make_bshd_map(&mk, k, B, N, H, d, 128) ||
+      !fa::make_bshd_map(&mv, v, B, N, H, d, 128))
+    return FA_ERR_LAUNCH;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return causal ? launch_fwd<128, true>(*di, mq, mk, mv, o, lse, B, H, N, scale, s)
+                  : launch_fwd<128, false>(*di, mq, mk, mv, o, lse, B, H, N, scale, s);
+  return causal ? launch_fwd<64, true>(*di, mq, mk, mv, o, lse, B, H, N, scale, s)
+                : launch_fwd<64, false>(*di, mq, mk, mv, o, lse, B, H, N, scale, s);
+}
+
+fa_status fa_get_status(void* stream) {
+  DeviceInfo* di = nullptr;
+  fa_status st = current_device(&di);
+  if (st != FA_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_DEVICE;
+  }
+  int word[2] = {0, 0};
+  const int zero[2] = {0, 0};
+  if (cudaMemcpyFromSymbol(word, g_fa_status, sizeof(word)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_fa_status, zero, sizeof(zero)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_DEVICE;
+  }
+  return word[0] == 0 ? FA_OK : static_cast<fa_status>(word[0]);
+}
+
+}  // extern "C"

@@ -1,0 +1,422 @@
+// fa_fwd_kernel.cuh -- fused exact-attention forward for sm_100a.
+//
+// One persistent CTA per SM walks a list of work tiles.  A tile is one
+// (batch, head) and a PAIR of 128-row query blocks; the pair shares one stream
+// of 128-key K/V tiles ("Flash Attention Explained", institutepm.com, "Tile the
+// input" / "Fuse into one kernel"; FlashAttention-2's partitioning over the
+// sequence dimension, same page, "Flash Attention 1, 2, and 3").
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax group 0: one thread per query row of block 0
+//   warps 4-7  softmax group 1: one thread per query row of block 1
+//   warp  8    TMA producer: Q blocks once per tile, then K_j, V_j into a ring of
+//              NSTAGE shared-memory slots (128-byte swizzle)
+//   warp  9    MMA issuer: S_i = Q_i K_j^T (both operands in shared memory) and
+//              O_i += P_i V_j (P read straight from tensor memory), accumulators
+//              in tensor memory; allocates / frees the 512 TMEM columns
+//
+// Tensor memory (512 columns x 128 lanes of 32 bit):
+//   [0,128)   S_0  (fp32 scores of block 0; P_0 overwrites its first 64 columns as bf16)
+//   [128,256) S_1
+//   [256, 256+D)     O_0 (fp32 accumulator)
+//   [256+D, 256+2D)  O_1
+//
+// Per K/V tile the MMA warp issues, in order, PV_0(j), S_0(j+1), PV_1(j), S_1(j+1):
+// while one softmax group works on its scores the tensor core computes the other
+// group's products (ping-pong).  tcgen05 ops issued by one thread complete in
+// order, so S_i(j+1) overwriting P_i(j) is safe, and the commit that signals
+// S_i(j+1) also guarantees PV_i(j) has finished.
+//
+// Online softmax ("Flash Attention Explained", "Compute softmax incrementally";
+// holysheep.ai review: running max and sum): scores are taken in base 2,
+// x = s * scale * log2(e).  Each row keeps a reference maximum m and a running
+// sum l of 2^(x - m).  m is only raised when the tile maximum exceeds it by more
+// than TAU (= 8, i.e. a factor 256); then l and the O accumulator are rescaled by
+// 2^(m_old - m_new).  Between raises the probabilities stay below 2^TAU, which
+// fp32 sums and bf16 P represent without loss, and O / l is unchanged because
+// numerator and denominator share the same reference.  Finally
+// O = O_acc / l and LSE = (m + log2 l) * ln 2.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+constexpr int kBM = 128;  // query rows per block
+constexpr int kBN = 128;  // keys per K/V tile
+constexpr int kFwdThreads = 320;
+constexpr float kTau = 8.0f;
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kChunks = D / 64;               // 64-column (128-byte) swizzle chunks per row
+  static constexpr int kTileBytes = 128 * D * 2;       // one 128-row bf16 tile
+  static constexpr int kChunkBytes = 128 * 128;        // one 128-row x 64-column chunk
+  static constexpr int kStages = (D == 128) ? 4 : 8;   // K/V ring slots
+  static constexpr uint32_t kOCol = 256;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+template <int D>
+struct __align__(1024) FwdSmem {
+  uint8_t q[2][FwdCfg<D>::kTileBytes];
+  uint8_t kv[FwdCfg<D>::kStages][FwdCfg<D>::kTileBytes];
+  uint64_t q_full[2];
+  uint64_t q_empty[2];
+  uint64_t kv_full[FwdCfg<D>::kStages];
+  uint64_t kv_empty[FwdCfg<D>::kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done[2];
+  uint64_t mma_drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// The k-th tile of CTA c: rounds of G tiles, walked forwards and backwards
+// alternately, so heavy and light tiles even out over the rounds.
+__device__ __forceinline__ int snake_tile(int c, int k, int G) {
+  return k * G + ((k & 1) ? (G - 1 - c) : c);
+}
+
+struct FwdTile {
+  int b, h, qb0;
+};
+
+// Tiles are ordered heaviest first (for causal attention the last query blocks
+// see the most keys), heads fastest, so concurrently running CTAs share K/V in L2.
+__device__ __forceinline__ FwdTile fwd_decode(int t, int BH, int H, int npairs) {
+  FwdTile ti;
+  const int p = npairs - 1 - t / BH;
+  const int bh = t % BH;
+  ti.b = bh / H;
+  ti.h = bh % H;
+  ti.qb0 = 2 * p;
+  return ti;
+}
+
+// Number of K/V tiles query block qb visits (0 if the block lies past the sequence).
+template <bool CAUSAL>
+__device__ __forceinline__ int fwd_nblocks(int qb, int nkb) {
+  if (qb >= nkb) return 0;
+  return CAUSAL ? qb + 1 : nkb;
+}
+
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int* status) {
+  // Used only while unwinding after an abort: ignores the abort flag, still bounded.
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(a, parity)) {
+    if (globaltimer_ns() - t0 > FA_WAIT_TIMEOUT_NS) {
+      atomicCAS(status, 0, 6);
+      return false;
+    }
+  }
+  return true;
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
+                  float* __restrict__ lse, int B, int H, int N, float scale_log2, int* status) {
+  using Cfg = FwdCfg<D>;
+  constexpr int NS = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                  ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nkb = (N + kBN - 1) / kBN;
+  const int npairs = (nkb + 1) / 2;
+  const int BH = B * H;
+  const int T = BH * npairs;
+
+  if (threadIdx.x == 0) {
+    sm.abort_flag = 0;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_empty[i], 1);
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], 128);
+      mbar_init(&sm.o_done[i], 1);
+    }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    mbar_init(&sm.mma_drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const WaitCtx wc{&sm.abort_flag, status, 1};
+      uint32_t it = 0, qcnt[2] = {0, 0};
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int t = snake_tile(blockIdx.x, k, gridDim.x);
+        if (t >= T) break;
+        const FwdTile ti = fwd_decode(t, BH, H, npairs);
+        const int n[2] = {fwd_nblocks<CAUSAL>(ti.qb0, nkb), fwd_nblocks<CAUSAL>(ti.qb0 + 1, nkb)};
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (n[i] == 0) continue;
+          ok = mbar_wait(&sm.q_empty[i], (qcnt[i] & 1) ^ 1, wc);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&sm.q_full[i], Cfg::kTileBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_4d(sm.q[i] + c * Cfg::kChunkBytes, &tm_q, &sm.q_full[i], c * 64, ti.h, (ti.qb0 + i) * kBM,
+                        ti.b);
+          ++qcnt[i];
+        }
+        const int nkv = n[0] > n[1] ? n[0] : n[1];
+        for (int j = 0; j < nkv && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv, ++it) {
+            const int s = it % NS;
+            ok = mbar_wait(&sm.kv_empty[s], ((it / NS) & 1) ^ 1, wc);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&sm.kv_full[s], Cfg::kTileBytes);
+            const CUtensorMap* m = kv ? &tm_v : &tm_k;
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_4d(sm.kv[s] + c * Cfg::kChunkBytes, m, &sm.kv_full[s], c * 64, ti.h, j * kBN, ti.b);
+          }
+        }
+      }
+      if (!ok) {
+        // Unwinding: wait (bounded) for the copies still in flight before the CTA exits.
+        for (uint32_t idx = (it > (uint32_t)NS ? it - NS : 0); idx < it; ++idx)
+          mbar_wait_drain(&sm.kv_full[idx % NS], (idx / NS) & 1, status);
+        for (int i = 0; i < 2; ++i)
+          if (qcnt[i] > 0) mbar_wait_drain(&sm.q_full[i], (qcnt[i] - 1) & 1, status);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const WaitCtx wc{&sm.abort_flag, status, 2};
+      constexpr uint32_t idesc_s = idesc_bf16(128, kBN, 0, 0);  // Q, K both K-major
+      constexpr uint32_t idesc_o = idesc_bf16(128, D, 0, 1);    // P from TMEM, V MN-major
+      const uint32_t q_addr[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+      const uint32_t kv_addr0 = smem_u32(sm.kv[0]);
+      uint32_t it = 0, qcnt[2] = {0, 0}, pcnt[2] = {0, 0};
+      bool ok = true;
+
+      auto issue_s = [&](int i, int slot) {
+        const uint32_t tS = tbase + i * 128;
+        const uint32_t kaddr = kv_addr0 + slot * Cfg::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * Cfg::kChunkBytes + (kk % 4) * 32;
+          umma_ss(tS, sdesc_sw128(q_addr[i] + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024), idesc_s,
+                  kk > 0);
+        }
+      };
+      auto issue_pv = [&](int i, int slot, uint32_t acc) {
+        const uint32_t tO = tbase + Cfg::kOCol + i * D;
+        const uint32_t tP = tbase + i * 128;
+        const uint32_t vaddr = kv_addr0 + slot * Cfg::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_ts(tO, tP + kk * 8, sdesc_sw128(vaddr + kk * 16 * 128, Cfg::kChunkBytes, 1024), idesc_o,
+                  (kk > 0) || acc);
+      };
+
+      for (int k = 0; ok; ++k) {
+        const int t = snake_tile(blockIdx.x, k, gridDim.x);
+        if (t >= T) break;
+        const FwdTile ti = fwd_decode(t, BH, H, npairs);
+        const int n[2] = {fwd_nblocks<CAUSAL>(ti.qb0, nkb), fwd_nblocks<CAUSAL>(ti.qb0 + 1, nkb)};
+        const int nkv = n[0] > n[1] ? n[0] : n[1];
+        for (int i = 0; i < 2 && ok; ++i)
+          if (n[i] > 0) ok = mbar_wait(&sm.q_full[i], qcnt[i] & 1, wc);
+        if (!ok) break;
+        // prologue: S_i(0)
+        const int sk0 = it % NS;
+        ok = mbar_wait(&sm.kv_full[sk0], (it / NS) & 1, wc);
+        if (!ok) break;
+        ++it;
+        tc_fence_after();
+        for (int i = 0; i < 2; ++i) {
+          if (n[i] == 0) continue;
+          issue_s(i, sk0);
+          umma_commit(&sm.s_full[i]);
+          if (n[i] == 1) umma_commit(&sm.q_empty[i]);
+        }
+        umma_commit(&sm.kv_empty[sk0]);
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int sv = it % NS;
+          ok = mbar_wait(&sm.kv_full[sv], (it / NS) & 1, wc);
+          if (!ok) break;
+          ++it;
+          int skn = -1;
+          if (j + 1 < nkv) {
+            skn = it % NS;
+            ok = mbar_wait(&sm.kv_full[skn], (it / NS) & 1, wc);
+            if (!ok) break;
+            ++it;
+          }
+          for (int i = 0; i < 2 && ok; ++i) {
+            if (j >= n[i]) continue;
+            ok = mbar_wait(&sm.p_full[i], pcnt[i] & 1, wc);
+            if (!ok) break;
+            ++pcnt[i];
+            tc_fence_after();
+            issue_pv(i, sv, j > 0);
+            if (j + 1 == n[i]) umma_commit(&sm.o_done[i]);
+            if (j + 1 < n[i]) {
+              issue_s(i, skn);
+              umma_commit(&sm.s_full[i]);
+              if (j + 2 == n[i]) umma_commit(&sm.q_empty[i]);
+            }
+          }
+          if (!ok) break;
+          umma_commit(&sm.kv_empty[sv]);
+          if (skn >= 0) umma_commit(&sm.kv_empty[skn]);
+        }
+        for (int i = 0; i < 2; ++i)
+          if (n[i] > 0) ++qcnt[i];
+      }
+      // Wait for every MMA issued to finish before the columns are freed.
+      umma_commit(&sm.mma_drain);
+      mbar_wait_drain(&sm.mma_drain, 0, status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax groups
+    const int g = warp >> 2;             // which query block of the pair
+    const int r = threadIdx.x & 127;     // row within the block == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tbase + g * 128 + lane_off;
+    const uint32_t tO = tbase + Cfg::kOCol + g * D + lane_off;
+    const WaitCtx wc{&sm.abort_flag, status, 3 + g};
+    uint32_t scnt = 0, ocnt = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int t = snake_tile(blockIdx.x, k, gridDim.x);
+      if (t >= T) break;
+      const FwdTile ti = fwd_decode(t, BH, H, npairs);
+      const int qb = ti.qb0 + g;
+      const int n = fwd_nblocks<CAUSAL>(qb, nkb);
+      if (n == 0) continue;
+      const int row = qb * kBM + r;
+      float m_ref = -INFINITY;
+      float l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[g], scnt & 1, wc));
+        if (!ok) break;
+        ++scnt;
+        tc_fence_after();
+        uint32_t s[kBN];
+        tmem_ld32(tS + 0, s + 0);
+        tmem_ld32(tS + 32, s + 32);
+        tmem_ld32(tS + 64, s + 64);
+        tmem_ld32(tS + 96, s + 96);
+        tmem_wait_ld();
+        const int k0 = j * kBN;
+        if (j == n - 1 && (CAUSAL || (N % kBN) != 0)) {
+          int lim = N - 1 - k0;                    // last valid key column of this tile
+          if (CAUSAL) lim = min(lim, row - k0);    // diagonal tile: key <= query
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (c > lim) s[c] = __float_as_uint(-INFINITY);
+        }
+        // row maximum: 8 independent chains, then combine
+        float mx8[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx8[x] = __uint_as_float(s[x]);
+#pragma unroll
+        for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(s[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float m_new = mx * scale_log2;
+        const bool raise = m_new > m_ref + kTau;
+        if (__any_sync(0xffffffffu, raise)) {
+          const float alpha = raise ? ex2_approx(m_ref - m_new) : 1.0f;
+          if (raise) {
+            l *= alpha;
+            m_ref = m_new;
+          }
+          if (j > 0) {
+            // PV(j-1) is complete: the commit that signalled S(j) covers it.
+#pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+              uint32_t o[32];
+              tmem_ld32(tO + c, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+              tmem_st32(tO + c, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        const float neg_m = -m_ref;
+        uint32_t p[kBN / 2];
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < kBN / 2; ++c) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * c]), scale_log2, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * c + 1]), scale_log2, neg_m));
+          rs[c & 3] += p0 + p1;
+          p[c] = pack_bf16x2(p0, p1);
+        }
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        tmem_st32(tS + 0, p);
+        tmem_st32(tS + 32, p + 32);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sm.p_full[g]);
+      }
+      if (!ok) break;
+      // epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done[g], ocnt & 1, wc));
+      if (!ok) break;
+      ++ocnt;
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const bool live = row < N;
+      __nv_bfloat16* orow = out + ((static_cast<int64_t>(ti.b) * N + row) * H + ti.h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + c, o);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          pk[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv_l, __uint_as_float(o[2 * x + 1]) * inv_l);
+        if (live) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        }
+      }
+      if (live) lse[(static_cast<int64_t>(ti.b) * H + ti.h) * N + row] = (m_ref + lg2_approx(l)) * kLn2;
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tbase, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,89 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library (libfa_b200.so).
+ *
+ * The operation is exact scaled-dot-product attention, O = softmax(scale * Q K^T) V,
+ * computed FlashAttention-style: Q, K and V are tiled into on-chip memory, the
+ * score tile, the online softmax (running row maximum and sum with rescaling) and
+ * the P.V product are fused in one kernel, and the N x N score matrix never
+ * reaches device memory ("Flash Attention Explained", institutepm.com, section
+ * "How Flash Attention Fixes It: Tiling and Recomputation"; holysheep.ai review,
+ * section "What Is Flash Attention and Why Does It Matter?").  The backward pass
+ * recomputes score tiles from the saved per-row log-sum-exp instead of storing
+ * the matrix (same page, "Recompute during backward pass").
+ *
+ * Tensor layout (the flash_attn_func interface of the holysheep.ai review,
+ * section "Implementing Flash Attention in Your Architecture"):
+ *   q, k, v, o, dO, dq, dk, dv : bf16, [B, N, H, d] contiguous (d innermost),
+ *                                element (b, n, h, x) at ((b*N + n)*H + h)*d + x.
+ *   lse                        : fp32, [B, H, N] contiguous, natural-log
+ *                                log-sum-exp of the scaled visible scores of each
+ *                                query row: lse = ln sum_j exp(scale * q.k_j).
+ * Queries and keys have the same length N.  causal = 1 lets query i see keys
+ * j <= i only ("Flash Attention vs Standard Attention", avichala.com, section
+ * "Engineering Perspective": autoregressive masking).  scale is the softmax
+ * scale; callers normally pass 1/sqrt(d), the default of the same interface.
+ *
+ * Pointers: every tensor pointer is a DEVICE pointer on the current CUDA device,
+ * 16-byte aligned (lse: 4-byte aligned), owned by the caller.  The library never
+ * allocates or frees device memory and keeps no per-call state; it caches the
+ * per-device kernel attributes and owns one small device status word.
+ *
+ * Execution: every call is asynchronous on `stream` (a cudaStream_t passed as
+ * void*; NULL = the legacy default stream).  Arguments are validated on the host
+ * BEFORE anything is enqueued; on any error nothing is launched.  Errors of the
+ * asynchronous execution surface on the caller's next synchronisation, and a
+ * kernel that had to give up on a bounded wait records FA_ERR_TIMEOUT in the
+ * status word read by fa_get_status().  No exception crosses the ABI and there
+ * is no fallback path: an unsupported case returns an error code.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* NULL pointer, B/H/N < 1, scale not finite and > 0, causal not 0/1, sizes overflow */
+  FA_ERR_UNSUPPORTED = 2, /* head dimension d other than 64 or 128 */
+  FA_ERR_ALIGNMENT = 3,   /* a tensor pointer not 16-byte aligned (lse: 4-byte) */
+  FA_ERR_DEVICE = 4,      /* no usable CUDA device, or the current device is not sm_100 */
+  FA_ERR_LAUNCH = 5,      /* kernel attribute setup or launch failed */
+  FA_ERR_TIMEOUT = 6,     /* a kernel abandoned a bounded wait (reported by fa_get_status) */
+  FA_ERR_WORKSPACE = 7    /* workspace pointer NULL or smaller than the required size */
+} fa_status;
+
+/* Library ABI version (this header: 1). */
+int fa_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(int status);
+
+/*
+ * Forward pass: o = softmax(scale * q k^T [masked]) v and lse per query row.
+ *   q, k, v : in,  bf16 [B, N, H, d]
+ *   o       : out, bf16 [B, N, H, d]
+ *   lse     : out, fp32 [B, H, N]
+ *   d       : 64 or 128
+ * Deterministic: the same inputs give bitwise-identical outputs.
+ * Device memory used beyond the arguments: none.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of the
+ * current device: FA_OK, or FA_ERR_TIMEOUT if a kernel gave up a bounded wait
+ * since the last call.  Returns FA_ERR_DEVICE if the stream or device reports a
+ * CUDA error.
+ */
+fa_status fa_get_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,64 @@
+"""Compare CUDA-path outputs with the fp64 oracle on the same seeded bf16 inputs.
+
+Tolerances (written here, used by every parity test):
+  O    : max |O_gpu - O_ref| <= 1e-2            (O is bf16)
+  LSE  : max |LSE_gpu - LSE_ref| / max(1, |LSE_ref|) <= 1e-3
+  dQ, dK, dV : max |g - g_ref| / max |g_ref| <= 2e-2, per tensor over the checked rows
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from exact_io_aware_93_b200.inputs import head_row_seed, sample_rows
+
+O_TOL = 1e-2
+LSE_TOL = 1e-3
+GRAD_TOL = 2e-2
+
+
+def _head(t: torch.Tensor, b: int, h: int) -> np.ndarray:
+    return t[b, :, h, :].to(torch.float64).numpy()
+
+
+def fwd_errors(inputs, o_gpu, lse_gpu, scale, causal, rows_per_head=None, seed=0, heads=None):
+    """Max errors of (O, LSE) over the checked rows of the given heads (default: all)."""
+    B, N, H, _ = inputs["q"].shape
+    o_gpu = o_gpu.cpu()
+    lse_gpu = lse_gpu.cpu()
+    heads = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    worst_o, worst_l, where = 0.0, 0.0, None
+    for b, h in heads:
+        rows = sample_rows(N, rows_per_head, head_row_seed(seed, b, h)).numpy()
+        o_ref, lse_ref = oracle.fwd_rows(_head(inputs["q"], b, h), _head(inputs["k"], b, h),
+                                         _head(inputs["v"], b, h), scale, causal, rows)
+        o_g = o_gpu[b, rows, h, :].to(torch.float64).numpy()
+        l_g = lse_gpu[b, h, rows].to(torch.float64).numpy()
+        eo = np.abs(o_g - o_ref)
+        el = np.abs(l_g - lse_ref) / np.maximum(1.0, np.abs(lse_ref))
+        if not np.all(np.isfinite(o_g)) or not np.all(np.isfinite(l_g)):
+            return float("inf"), float("inf"), (b, h, "non-finite")
+        if eo.max() > worst_o:
+            r = int(np.unravel_index(eo.argmax(), eo.shape)[0])
+            worst_o, where = float(eo.max()), (b, h, int(rows[r]))
+        worst_l = max(worst_l, float(el.max()))
+    return worst_o, worst_l, where
+
+
+def grad_errors(inputs, grads_gpu, scale, causal, heads_full, heads_sampled):
+    """Relative max errors of dQ, dK, dV: full heads, plus (b, h, rows) sampled heads."""
+    B, N, H, _ = inputs["q"].shape
+    num = {"dq": 0.0, "dk": 0.0, "dv": 0.0}
+    den = {"dq": 0.0, "dk": 0.0, "dv": 0.0}
+    jobs = [(b, h, None) for b, h in heads_full] + list(heads_sampled)
+    for b, h, rows in jobs:
+        rows_np = np.arange(N) if rows is None else np.asarray(rows)
+        dq, _, dk, dv = oracle.bwd_rows(_head(inputs["q"], b, h), _head(inputs["k"], b, h),
+                                        _head(inputs["v"], b, h), _head(inputs["do"], b, h),
+                                        scale, causal, rows_np, rows_np)
+        for name, ref in (("dq", dq), ("dk", dk), ("dv", dv)):
+            got = grads_gpu[name][b, rows_np, h, :].to(torch.float64).cpu().numpy()
+            num[name] = max(num[name], float(np.abs(got - ref).max()))
+            den[name] = max(den[name], float(np.abs(ref).max()))
+    return {n: num[n] / max(den[n], 1e-30) for n in num}

@@ -1,0 +1,83 @@
+"""The C ABI library: builds, loads and exports every declared symbol; host-side
+argument validation returns the documented codes without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_93_b200 import build as fabuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
+
+
+def declared_functions():
+    names = []
+    for path in HEADERS:
+        text = open(path).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w\s\*]*?\b(fa_\w+)\s*\(", text, flags=re.M):
+            names.append(m.group(1))
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = fabuild.build()
+    return ctypes.CDLL(path)
+
+
+def test_headers_declare_entry_points():
+    names = declared_functions()
+    assert "fa_fwd" in names and "fa_get_status" in names and "fa_status_string" in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/*.h but not exported"
+
+
+def test_status_strings(lib):
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_status_string.argtypes = [ctypes.c_int]
+    assert lib.fa_status_string(0) == b"FA_OK"
+    assert lib.fa_status_string(6) == b"FA_ERR_TIMEOUT"
+    assert lib.fa_status_string(99) == b"FA_ERR_UNKNOWN"
+    assert lib.fa_abi_version() == 1
+
+
+def _fwd(lib, q=0x10000, k=0x10000, v=0x10000, o=0x10000, lse=0x10000, B=1, H=1, N=16, d=64,
+         scale=0.125, causal=0):
+    vp = ctypes.c_void_p
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                           ctypes.c_float, ctypes.c_int, vp]
+    lib.fa_fwd.restype = ctypes.c_int
+    return lib.fa_fwd(vp(q), vp(k), vp(v), vp(o), vp(lse), B, H, N, d, ctypes.c_float(scale), causal, None)
+
+
+def test_fwd_validation_codes(lib):
+    assert _fwd(lib, q=0) == 1
+    assert _fwd(lib, lse=0) == 1
+    assert _fwd(lib, B=0) == 1
+    assert _fwd(lib, N=0) == 1
+    assert _fwd(lib, H=-1) == 1
+    assert _fwd(lib, scale=0.0) == 1
+    assert _fwd(lib, scale=float("nan")) == 1
+    assert _fwd(lib, scale=float("inf")) == 1
+    assert _fwd(lib, causal=2) == 1
+    assert _fwd(lib, d=96) == 2
+    assert _fwd(lib, d=256) == 2
+    assert _fwd(lib, q=0x10008) == 3
+    assert _fwd(lib, o=0x10004) == 3
+    assert _fwd(lib, lse=0x10002) == 3
+    assert _fwd(lib, B=1 << 20, H=1 << 10, N=1 << 20, d=128) == 1
+
+
+def test_fwd_without_gpu_reports_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is visible: the device check passes")
+    assert _fwd(lib) == 4
