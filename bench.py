@@ -1,0 +1,347 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200: one step = fa_fwd + fa_bwd.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Workload (default): causal, B=2, H=16, N=8192, d=128, bf16 -- the forward +
+recompute-backward configuration.  Inputs are seeded synthetic N(0,1) bf16
+(``exact_io_aware_93_b200.inputs``), resident in HBM before the timed region.
+Q, K, V, dO, O together exceed the 126 MB L2, so L2 is not flushed between steps.
+
+Prints ONE JSON line (rank 0).  ``value`` is whole-job TFLOPS under the FLOP
+convention forward = 4*B*H*N^2*d (halved when causal), backward = 2.5x forward,
+summed over all ranks.  With N > 1 (torchrun) every rank runs the same workload
+on its own GPU (independent replicas, weak scaling, no data-path collective);
+the time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the slow, plain definition the
+parity tests use) on the host cores, each step one full head of the same
+workload (forward and backward), and prints the same JSON line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_io_aware_93_b200.accounting import bwd_flops, fwd_bytes, fwd_flops  # noqa: E402
+from exact_io_aware_93_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "attention fwd/bwd TFLOPS and % of B200 dense-bf16 peak, causal N=2K–128K"
+DEFAULT_WORKLOAD = "causal_fwdbwd_b2_h16_n8192_d128"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), \
+            float(p["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fa_bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}", "--format=csv,noheader",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1].split()[0]))
+                    smax.append(float(parts[2].split()[0]))
+                    power.append(float(parts[3].split()[0]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        loaded = [s for s in sm if smax and s > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def _step_fn(api, t, w, with_bwd, events=None):
+    """One pass of the hot path: fa_fwd then (if available) fa_bwd, on the current stream."""
+    def step():
+        if events is not None:
+            events["fwd"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+            events["fwd"][-1][0].record()
+        api.fwd(t["q"], t["k"], t["v"], causal=w.causal, out=t["o"], lse=t["lse"])
+        if events is not None:
+            events["fwd"][-1][1].record()
+        if with_bwd:
+            if events is not None:
+                events["bwd"].append((torch.cuda.Event(enable_timing=True),
+                                      torch.cuda.Event(enable_timing=True)))
+                events["bwd"][-1][0].record()
+            api.bwd(t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], causal=w.causal,
+                    dq=t["dq"], dk=t["dk"], dv=t["dv"], workspace=t["ws"])
+            if events is not None:
+                events["bwd"][-1][1].record()
+    return step
+
+
+def cpu_sample(w, heads: int, threads: int):
+    """Time the fp64 oracle on `heads` full heads of workload w (forward and backward)."""
+    import oracle
+    oracle.oracle_threads(threads)
+    inp = make_inputs(1, heads, w.N, w.d, w.seed, with_do=with_bwd_available())
+    t0 = time.perf_counter()
+    flops = 0.0
+    for h in range(heads):
+        q, k, v = (inp[n][0, :, h].double().numpy() for n in ("q", "k", "v"))
+        oracle.fwd_rows(q, k, v, w.scale, w.causal)
+        flops += fwd_flops(1, 1, w.N, w.d, w.causal)
+        if with_bwd_available():
+            do = inp["do"][0, :, h].double().numpy()
+            oracle.bwd_rows(q, k, v, do, w.scale, w.causal)
+            flops += bwd_flops(1, 1, w.N, w.d, w.causal)
+    dt = time.perf_counter() - t0
+    return flops, dt
+
+
+def with_bwd_available() -> bool:
+    try:
+        from exact_io_aware_93_b200 import api
+        return hasattr(api.lib(), "fa_bwd") and hasattr(api, "bwd")
+    except (FileNotFoundError, OSError):
+        return False
+
+
+def run_reference(args, w):
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return 0
+    threads = len(os.sched_getaffinity(0))
+    heads = 1
+    times = []
+    flops_step = 0.0
+    for i in range(args.warmup + args.steps):
+        flops_step, dt = cpu_sample(w, heads, threads)
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = flops_step * len(times) / total / 1e12
+    sample = (f"{heads} full head(s) (b=0, h=0) of {w.name}: forward"
+              + (" and backward" if with_bwd_available() else "") + " of every row, fp64")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w):
+    world, rank, local = _dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from exact_io_aware_93_b200 import api
+    dev = torch.device("cuda", torch.cuda.current_device())
+    with_bwd = with_bwd_available()
+
+    inp = make_inputs(w.B, w.H, w.N, w.d, w.seed, with_do=True, peaked=w.peaked)
+    t = {n: inp[n].to(dev) for n in ("q", "k", "v", "do")}
+    t["o"] = torch.empty_like(t["q"])
+    t["lse"] = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    if with_bwd:
+        t["dq"], t["dk"], t["dv"] = (torch.empty_like(t["q"]) for _ in range(3))
+        t["ws"] = torch.empty(api.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    in_bytes = sum(t[n].numel() * t[n].element_size() for n in ("q", "k", "v", "do"))
+
+    step = _step_fn(api, t, w, with_bwd)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if api.get_status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    # ---------------- device-timed region
+    events = {"fwd": [], "bwd": []}
+    tstep = _step_fn(api, t, w, with_bwd, events)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        tstep()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in events["fwd"])
+    bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in events["bwd"]) if events["bwd"] else None
+    status = api.get_status()
+
+    # ---------------- end-to-end through the public API: pinned host in, results back
+    host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "do")}
+    out_host = {n: torch.empty(t[n].shape, dtype=t[n].dtype).pin_memory()
+                for n in (["o", "lse"] + (["dq", "dk", "dv"] if with_bwd else []))}
+    d2h_bytes = sum(x.numel() * x.element_size() for x in out_host.values())
+    e2e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        for n in ("q", "k", "v", "do"):
+            t[n].copy_(host[n], non_blocking=True)
+        step()
+        for n, x in out_host.items():
+            x.copy_(t[n], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+
+    if world > 1:
+        tt = torch.tensor([ms, e2e_ms, fwd_ms, bwd_ms or 0.0], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, e2e_ms, fwd_ms, bwd_ms = (float(x) for x in tt.tolist())
+        bwd_ms = bwd_ms if with_bwd else None
+
+    ff = fwd_flops(w.B, w.H, w.N, w.d, w.causal)
+    fb = bwd_flops(w.B, w.H, w.N, w.d, w.causal) if with_bwd else 0.0
+    step_flops = ff + fb
+    value = world * step_flops / (ms * 1e-3) / 1e12
+    e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+    peak, peak_sus, hbm, peak_kind = _peaks()
+    fwd_tf = ff / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = fb / (bwd_ms * 1e-3) / 1e12 if with_bwd else None
+    # dominant kernel: the one with the larger share of the step
+    if with_bwd and bwd_ms > fwd_ms:
+        dom = {"kernel": "fa_bwd (pre + main + post)", "achieved": bwd_tf, "ms": bwd_ms}
+    else:
+        dom = {"kernel": "fa_fwd_kernel", "achieved": fwd_tf, "ms": fwd_ms}
+    roofline = {"bound": "tensor", "achieved": dom["achieved"], "peak": peak, "unit": "TFLOP/s",
+                "frac": dom["achieved"] / peak, "traffic": None, "kernel": dom["kernel"],
+                "peak_kind": f"{peak_kind} bf16 burst (cuBLAS 8192^3)",
+                "frac_of_sustained": dom["achieved"] / peak_sus,
+                "fwd_alg_bytes": fwd_bytes(w.B, w.H, w.N, w.d)}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"not flushed: inputs {in_bytes / 1e6:.0f} MB > L2 {L2_BYTES / 1e6:.0f} MB",
+                   "step": "fa_fwd + fa_bwd" if with_bwd else "fa_fwd only (backward not built)"},
+        "fwd_tflops": fwd_tf, "fwd_ms": fwd_ms, "bwd_tflops": bwd_tf, "bwd_ms": bwd_ms,
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": d2h_bytes, "ms_per_step": e2e_ms, "steps": e2e_steps},
+        "gpu_launches": args.steps * (1 + (3 if with_bwd else 0)),
+        "clocks": clk,
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = len(os.sched_getaffinity(0))
+        heads = 4
+        cflops, cdt = cpu_sample(w, heads, threads)
+        line["cpu_baseline"] = {
+            "value": cflops / cdt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{heads} full heads of {w.name} (forward" + (" + backward" if with_bwd else "")
+                      + f", fp64), {cdt:.1f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -6,7 +6,7 @@
 // input" / "Fuse into one kernel"; FlashAttention-2's partitioning over the
 // sequence dimension, same page, "Flash Attention 1, 2, and 3").
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax group 0: one thread per query row of block 0
 //   warps 4-7  softmax group 1: one thread per query row of block 1
 //   warp  8    TMA producer: Q blocks once per tile, then K_j, V_j into a ring of
@@ -14,6 +14,10 @@
 //   warp  9    MMA issuer: S_i = Q_i K_j^T (both operands in shared memory) and
 //              O_i += P_i V_j (P read straight from tensor memory), accumulators
 //              in tensor memory; allocates / frees the 512 TMEM columns
+//   warps 10-11 idle
+// Registers: launched at 168 per thread (384 x 168 = 64512); the softmax warpgroups
+// raise theirs to 200 and the producer/MMA warpgroup drops to 96:
+// 2 x 128 x 200 + 128 x 96 = 63488 <= 64512.
 //
 // Tensor memory (512 columns x 128 lanes of 32 bit):
 //   [0,128)   S_0  (fp32 scores of block 0; P_0 overwrites its first 64 columns as bf16)
@@ -34,8 +38,10 @@
 // than TAU (= 8, i.e. a factor 256); then l and the O accumulator are rescaled by
 // 2^(m_old - m_new).  Between raises the probabilities stay below 2^TAU, which
 // fp32 sums and bf16 P represent without loss, and O / l is unchanged because
-// numerator and denominator share the same reference.  Finally
-// O = O_acc / l and LSE = (m + log2 l) * ln 2.
+// numerator and denominator share the same reference.  Two sums are kept: l of
+// the fp32 probabilities (for the log-sum-exp) and lr of the bf16-rounded
+// probabilities that actually enter the P.V product, so that O = O_acc / lr is
+// an exact convex combination of value rows.  Finally LSE = (m + log2 l) * ln 2.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -44,7 +50,11 @@ namespace fa {
 
 constexpr int kBM = 128;  // query rows per block
 constexpr int kBN = 128;  // keys per K/V tile
-constexpr int kFwdThreads = 320;
+constexpr int kFwdThreads = 384;
+constexpr uint32_t kFwdRegsSoftmax = 200;
+constexpr uint32_t kFwdRegsOther = 96;
+static_assert(2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsOther <= kFwdThreads * 168,
+              "register split exceeds the launch allocation");
 constexpr float kTau = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
@@ -163,6 +173,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
 
+  if (warp >= 8) regs_decrease<kFwdRegsOther>();
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -296,8 +307,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_wait_drain(&sm.mma_drain, 0, status);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax groups
+    regs_increase<kFwdRegsSoftmax>();
     const int g = warp >> 2;             // which query block of the pair
     const int r = threadIdx.x & 127;     // row within the block == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -315,7 +327,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (n == 0) continue;
       const int row = qb * kBM + r;
       float m_ref = -INFINITY;
-      float l = 0.f;
+      float l = 0.f;    // sum of 2^(x - m) in fp32: the log-sum-exp
+      float lr = 0.f;   // sum of the same weights rounded to bf16: normalises O
       for (int j = 0; j < n; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[g], scnt & 1, wc));
         if (!ok) break;
@@ -335,20 +348,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (c > lim) s[c] = __float_as_uint(-INFINITY);
         }
-        // row maximum: 8 independent chains, then combine
+        // row maximum: 8 independent chains of three-input max, then combine
         float mx8[8];
 #pragma unroll
-        for (int x = 0; x < 8; ++x) mx8[x] = __uint_as_float(s[x]);
+        for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(__uint_as_float(s[x]), __uint_as_float(s[x + 8]));
 #pragma unroll
-        for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(s[c]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int c = 16; c < kBN; c += 16)
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            mx8[x] = fmax3(mx8[x], __uint_as_float(s[c + x]), __uint_as_float(s[c + 8 + x]));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
         const float m_new = mx * scale_log2;
         const bool raise = m_new > m_ref + kTau;
         if (__any_sync(0xffffffffu, raise)) {
           const float alpha = raise ? ex2_approx(m_ref - m_new) : 1.0f;
           if (raise) {
             l *= alpha;
+            lr *= alpha;
             m_ref = m_new;
           }
           if (j > 0) {
@@ -365,17 +382,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_wait_st();
           }
         }
-        const float neg_m = -m_ref;
+        const float2 sl2 = make_float2(scale_log2, scale_log2);
+        const float2 nm2 = make_float2(-m_ref, -m_ref);
         uint32_t p[kBN / 2];
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 se[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 sr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < kBN / 2; ++c) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * c]), scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * c + 1]), scale_log2, neg_m));
-          rs[c & 3] += p0 + p1;
+          const float2 x = ffma2(make_float2(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sl2, nm2);
+          const float p0 = ex2_approx(x.x);
+          const float p1 = ex2_approx(x.y);
           p[c] = pack_bf16x2(p0, p1);
+          se[c & 1] = fadd2(se[c & 1], make_float2(p0, p1));
+          // the bf16 weights the P.V product actually uses: O = O_acc / lr is an exact
+          // convex combination of value rows (the rounding of a dominant weight cancels)
+          sr[c & 1] = fadd2(sr[c & 1], make_float2(__uint_as_float(p[c] << 16),
+                                                   __uint_as_float(p[c] & 0xffff0000u)));
         }
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        l += (se[0].x + se[0].y) + (se[1].x + se[1].y);
+        lr += (sr[0].x + sr[0].y) + (sr[1].x + sr[1].y);
         tmem_st32(tS + 0, p);
         tmem_st32(tS + 32, p + 32);
         tmem_wait_st();
@@ -388,7 +413,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (!ok) break;
       ++ocnt;
       tc_fence_after();
-      const float inv_l = 1.0f / l;
+      const float inv_l = 1.0f / lr;
       const bool live = row < N;
       __nv_bfloat16* orow = out + ((static_cast<int64_t>(ti.b) * N + row) * H + ti.h) * D;
 #pragma unroll 1

@@ -40,8 +40,11 @@ def fwd_errors(inputs, o_gpu, lse_gpu, scale, causal, rows_per_head=None, seed=0
         if not np.all(np.isfinite(o_g)) or not np.all(np.isfinite(l_g)):
             return float("inf"), float("inf"), (b, h, "non-finite")
         if eo.max() > worst_o:
-            r = int(np.unravel_index(eo.argmax(), eo.shape)[0])
-            worst_o, where = float(eo.max()), (b, h, int(rows[r]))
+            r, c = (int(x) for x in np.unravel_index(eo.argmax(), eo.shape))
+            o_ref_bf16 = float(torch.tensor(o_ref[r, c]).to(torch.bfloat16).double())
+            worst_o = float(eo.max())
+            where = dict(b=b, h=h, row=int(rows[r]), col=c, o_ref=float(o_ref[r, c]),
+                         o_gpu=float(o_g[r, c]), err_vs_bf16_ref=abs(float(o_g[r, c]) - o_ref_bf16))
         worst_l = max(worst_l, float(el.max()))
     return worst_o, worst_l, where
 
