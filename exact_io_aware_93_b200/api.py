@@ -55,12 +55,11 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd.restype = i
     L.fa_get_status.argtypes = [vp]
     L.fa_get_status.restype = i
-    if hasattr(L, "fa_bwd"):
-        L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
-        L.fa_bwd_workspace_size.restype = ctypes.c_size_t
-        L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
-                             i, i, i, i, f, i, vp]
-        L.fa_bwd.restype = i
+    L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    L.fa_bwd_workspace_size.restype = ctypes.c_size_t
+    L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                         i, i, i, i, f, i, vp]
+    L.fa_bwd.restype = i
     _lib = L
     return L
 
@@ -112,6 +111,41 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     if st != 0:
         raise FAError(st, "fa_fwd")
     return out, lse
+
+
+def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    """Bytes of device workspace ``fa_bwd`` needs (fp32 dQ accumulator and row sums D)."""
+    return int(lib().fa_bwd_workspace_size(B, H, N, d))
+
+
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, do: torch.Tensor,
+        lse: torch.Tensor, causal: bool = False, scale: float | None = None,
+        dq: torch.Tensor | None = None, dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
+        workspace: torch.Tensor | None = None):
+    """(dQ, dK, dV) of L = sum(O * dO) via ``fa_bwd`` (score tiles recomputed from LSE)."""
+    validate_inputs(q, k, v)
+    for name, t in (("o", o), ("do", do)):
+        if t.shape != q.shape or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name} must be a contiguous bf16 tensor shaped like q")
+    B, N, H, d = q.shape
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                      workspace.data_ptr(), ws_bytes, B, H, N, d, ctypes.c_float(scale),
+                      int(bool(causal)), _stream_ptr(q))
+    if st != 0:
+        raise FAError(st, "fa_bwd")
+    return dq, dk, dv
 
 
 def get_status(device: torch.device | None = None) -> int:

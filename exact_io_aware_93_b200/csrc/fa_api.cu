@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "../../include/fa.h"
+#include "fa_bwd_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 #include "tma_host.h"
 
@@ -22,10 +23,24 @@ struct DeviceInfo {
   int sm_count = 0;
   int* status = nullptr;
   bool fwd_attr[2][2] = {{false, false}, {false, false}};  // [d==128][causal]
+  bool bwd_attr[2][2] = {{false, false}, {false, false}};
 };
 DeviceInfo g_dev[kMaxDevices];
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The warp-specialised kernels move registers between warpgroups with setmaxnreg; the
+// split is computed for a launch at exactly fa::kLaunchRegs registers per thread.
+// Refuse to launch a build whose register count differs.
+template <typename K>
+bool launch_regs_ok(K kern) {
+  cudaFuncAttributes a;
+  if (cudaFuncGetAttributes(&a, kern) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.numRegs == static_cast<int>(fa::kLaunchRegs);
+}
 
 fa_status current_device(DeviceInfo** out) {
   int dev = -1;
@@ -74,7 +89,8 @@ fa_status launch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   const int smem = static_cast<int>(sizeof(fa::FwdSmem<D>)) + 1024;
   bool& attr = di.fwd_attr[D == 128][CAUSAL];
   if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    if (!launch_regs_ok(kern) ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
       cudaGetLastError();
       return FA_ERR_LAUNCH;
     }
@@ -86,6 +102,46 @@ fa_status launch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   const float scale_log2 = scale * 1.4426950408889634f;
   kern<<<grid, fa::kFwdThreads, smem, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, B, H, N,
                                                  scale_log2, di.status);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+size_t bwd_ws_bytes(int B, int H, int N, int d) {
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return rows * static_cast<size_t>(d) * 4 + rows * 4;  // fp32 dQ accumulator + fp32 D
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& mdo, const void* o, const void* dO, const float* lse, void* dq, void* dk,
+                     void* dv, void* ws, int B, int H, int N, float scale, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(B) * H * N;
+  float* dq_acc = static_cast<float*>(ws);
+  float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + rows * D * 4);
+  const int64_t ew_threads = rows * (D / 8);
+  const unsigned ew_blocks = static_cast<unsigned>((ew_threads + 255) / 256);
+  fa::fa_bwd_pre_kernel<D><<<ew_blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                          static_cast<const __nv_bfloat16*>(dO), dsum, dq_acc, B,
+                                                          H, N);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  auto kern = fa::fa_bwd_main_kernel<D, CAUSAL>;
+  const int smem = static_cast<int>(sizeof(fa::BwdSmem<D>));
+  bool& attr = di.bwd_attr[D == 128][CAUSAL];
+  if (!attr) {
+    if (!launch_regs_ok(kern) ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    attr = true;
+  }
+  const int nkb = (N + 127) / 128;
+  kern<<<B * H * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, lse, dsum, dq_acc,
+                                                        static_cast<__nv_bfloat16*>(dk),
+                                                        static_cast<__nv_bfloat16*>(dv), B, H, N, scale, di.status);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  fa::fa_bwd_post_kernel<D><<<ew_blocks, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), B, H, N,
+                                                           scale);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
 }
@@ -130,6 +186,38 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                   : launch_fwd<128, false>(*di, mq, mk, mv, o, lse, B, H, N, scale, s);
   return causal ? launch_fwd<64, true>(*di, mq, mk, mv, o, lse, B, H, N, scale, s)
                 : launch_fwd<64, false>(*di, mq, mk, mv, o, lse, B, H, N, scale, s);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  return bwd_ws_bytes(B, H, N, d);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                 float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGNMENT;
+  if (workspace == nullptr || workspace_bytes < bwd_ws_bytes(B, H, N, d)) return FA_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return FA_ERR_ALIGNMENT;
+  if (static_cast<long long>(B) * H * ((static_cast<long long>(N) + 127) / 128) > INT32_MAX) return FA_ERR_INVALID_ARG;
+  DeviceInfo* di = nullptr;
+  st = current_device(&di);
+  if (st != FA_OK) return st;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!fa::make_bshd_map(&mq, q, B, N, H, d, 128) || !fa::make_bshd_map(&mk, k, B, N, H, d, 128) ||
+      !fa::make_bshd_map(&mv, v, B, N, H, d, 128) || !fa::make_bshd_map(&mdo, dO, B, N, H, d, 128))
+    return FA_ERR_LAUNCH;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return causal ? launch_bwd<128, true>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s)
+                  : launch_bwd<128, false>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s);
+  return causal ? launch_bwd<64, true>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s)
+                : launch_bwd<64, false>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s);
 }
 
 fa_status fa_get_status(void* stream) {

@@ -1,0 +1,449 @@
+// fa_bwd_kernel.cuh -- exact-attention backward for sm_100a, recomputing score tiles
+// from the saved log-sum-exp instead of storing the N x N matrix ("Flash Attention
+// Explained", institutepm.com, "Recompute during backward pass"; "What Is Flash
+// Attention?", bestllmfor.com, "How Flash Attention works": recomputation).
+//
+// Gradients of L = sum(O * dO) with P = softmax(scale * Q K^T):
+//   dV = P^T dO,   dP = dO V^T,   dS = P o (dP - D),   D_i = sum_x dO_ix O_ix,
+//   dK = scale * dS^T Q,   dQ = scale * dS K.
+// D_i equals the Jacobian row constant sum_t P_it dP_it because O_i = sum_t P_it v_t.
+//
+// Three kernels, one stream:
+//   fa_bwd_pre  : D_i (fp32) and zeroing of the fp32 dQ accumulator (memory bound)
+//   fa_bwd_main : one CTA per (batch, head, 128-key block j); K_j and V_j stay in shared
+//                 memory while 128-query blocks i (i >= j when causal) stream through:
+//                   S^T  = K_j Q_i^T        (tcgen05, both operands in shared memory)
+//                   dP^T = V_j dO_i^T
+//                   P^T  = 2^(S^T * scale * log2 e - LSE_i * log2 e)   (one thread per key)
+//                   dS^T = P^T o (dP^T - D_i)
+//                   dV_j += P^T dO_i        (A operand P^T read from tensor memory)
+//                   dK_j += dS^T Q_i        (A operand dS^T read from tensor memory)
+//                   dQ_i  = dS K_j          (dS written to shared memory, 128-byte swizzle)
+//                 and a drain warpgroup adds each dQ_i tile into the fp32 accumulator with
+//                 vector reductions; dK_j, dV_j are written once at the end.
+//   fa_bwd_post : dQ = bf16(scale * accumulator)
+//
+// Tensor memory (512 columns):
+//   [0,128)   S^T  (fp32; P^T overwrites its first 64 columns as bf16)
+//   [128,256) dP^T (fp32; dS^T overwrites its first 64 columns; then dQ_i, fp32, D columns)
+//   [256,256+D) dV_j accumulator,  [384,384+D) dK_j accumulator
+//
+// Warp roles (384 threads): warps 0-3 key rows (P, dS, final dK/dV), warps 4-7 dQ drain,
+// warp 8 loads (TMA for tiles, plain loads for LSE and D), warp 9 issues MMAs.
+#pragma once
+
+#include "fa_fwd_kernel.cuh"
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+constexpr int kBwdThreads = 384;
+constexpr uint32_t kBwdRegsKey = 224;
+constexpr uint32_t kBwdRegsDrain = 128;
+constexpr uint32_t kBwdRegsOther = 96;
+static_assert(128 * (kBwdRegsKey + kBwdRegsDrain + kBwdRegsOther) <= kBwdThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kChunkBytes = 128 * 128;
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColDP = 128;
+  static constexpr uint32_t kColDV = 256;
+  static constexpr uint32_t kColDK = 384;
+};
+
+template <int D>
+struct __align__(1024) BwdSmem {
+  uint8_t k[BwdCfg<D>::kTileBytes];
+  uint8_t v[BwdCfg<D>::kTileBytes];
+  uint8_t q[2][BwdCfg<D>::kTileBytes];
+  uint8_t dO[2][BwdCfg<D>::kTileBytes];
+  uint8_t ds[128 * 128 * 2];  // dS (queries x keys), MN-major A operand of dQ = dS K
+  float lse2[2][128];         // LSE * log2(e) of the query block (+inf past the sequence)
+  float dd[2][128];           // D of the query block
+  uint64_t kv_full;
+  uint64_t qd_full[2];
+  uint64_t qd_empty[2];
+  uint64_t s_full;
+  uint64_t dp_full;
+  uint64_t ds_ready;
+  uint64_t dq_full;
+  uint64_t dq_free;
+  uint64_t acc_done;
+  uint64_t mma_drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// ---------------------------------------------------------------- pre
+// D[b,h,n] = sum_x dO[b,n,h,x] * O[b,n,h,x]; zero the dQ accumulator rows.
+// One group of D/8 threads per row, 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                         const __nv_bfloat16* __restrict__ dout,
+                                                         float* __restrict__ dsum, float* __restrict__ dq_acc,
+                                                         int B, int H, int N) {
+  constexpr int TPR = D / 8;  // threads per row
+  const int64_t rows = static_cast<int64_t>(B) * H * N;
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TPR;
+  const int part = threadIdx.x % TPR;
+  float acc = 0.f;
+  if (row < rows) {
+    const int64_t bh = row / N;
+    const int n = static_cast<int>(row % N);
+    const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
+    const int64_t off = ((static_cast<int64_t>(b) * N + n) * H + h) * D + part * 8;
+    const uint4 ov = *reinterpret_cast<const uint4*>(o + off);
+    const uint4 dv = *reinterpret_cast<const uint4*>(dout + off);
+    const __nv_bfloat162* op = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __nv_bfloat162* dp = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const float2 a = __bfloat1622float2(op[x]);
+      const float2 c = __bfloat1622float2(dp[x]);
+      acc = fmaf(a.x, c.x, acc);
+      acc = fmaf(a.y, c.y, acc);
+    }
+    float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int s = TPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (row < rows && part == 0) dsum[row] = acc;
+}
+
+// ---------------------------------------------------------------- post
+// dQ[b,n,h,:] = bf16(scale * acc[b,h,n,:]), 8 elements per thread.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restrict__ dq_acc,
+                                                          __nv_bfloat16* __restrict__ dq, int B, int H, int N,
+                                                          float scale) {
+  constexpr int TPR = D / 8;
+  const int64_t rows = static_cast<int64_t>(B) * H * N;
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TPR;
+  const int part = threadIdx.x % TPR;
+  if (row >= rows) return;
+  const int64_t bh = row / N;
+  const int n = static_cast<int>(row % N);
+  const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
+  const float4* a = reinterpret_cast<const float4*>(dq_acc + row * D + part * 8);
+  const float4 a0 = a[0], a1 = a[1];
+  uint4 r;
+  r.x = pack_bf16x2(a0.x * scale, a0.y * scale);
+  r.y = pack_bf16x2(a0.z * scale, a0.w * scale);
+  r.z = pack_bf16x2(a1.x * scale, a1.y * scale);
+  r.w = pack_bf16x2(a1.z * scale, a1.w * scale);
+  *reinterpret_cast<uint4*>(dq + ((static_cast<int64_t>(b) * N + n) * H + h) * D + part * 8) = r;
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+// ---------------------------------------------------------------- main
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const float* __restrict__ lse, const float* __restrict__ dsum,
+                       float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                       int B, int H, int N, float scale, int* status) {
+  using Cfg = BwdCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0) {  // the layout relies on a 1 KB aligned base
+    if (threadIdx.x == 0) atomicCAS(status, 0, 5);
+    return;
+  }
+  BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nkb = (N + 127) / 128;
+  const int BH = B * H;
+  // heavy key blocks first: with causal masking block j meets nkb - j query blocks
+  const int j = blockIdx.x / BH;
+  const int bh = blockIdx.x % BH;
+  const int b = bh / H, h = bh % H;
+  const int i0 = CAUSAL ? j : 0;
+  const int ni = nkb - i0;
+
+  if (threadIdx.x == 0) {
+    sm.abort_flag = 0;
+    mbar_init(&sm.kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.qd_full[s], 2);  // expect-tx arrive + arrive after LSE / D stores
+      mbar_init(&sm.qd_empty[s], 1);
+    }
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.dp_full, 1);
+    mbar_init(&sm.ds_ready, 128);
+    mbar_init(&sm.dq_full, 1);
+    mbar_init(&sm.dq_free, 128);
+    mbar_init(&sm.acc_done, 1);
+    mbar_init(&sm.mma_drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+
+  // Each warpgroup's setmaxnreg sits at the top of the branch holding all of that
+  // warpgroup's code, so every instruction after it is compiled within the new limit.
+  if (warp >= 8) {
+    regs_set<kLaunchRegs, kBwdRegsOther>();
+  if (warp == 8) {
+    // ------------------------------------------------------------ loads
+    const WaitCtx wc{&sm.abort_flag, status, 11};
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(&sm.kv_full, 2 * Cfg::kTileBytes);
+      for (int c = 0; c < Cfg::kChunks; ++c) {
+        tma_load_4d(sm.k + c * Cfg::kChunkBytes, &tm_k, &sm.kv_full, c * 64, h, j * 128, b);
+        tma_load_4d(sm.v + c * Cfg::kChunkBytes, &tm_v, &sm.kv_full, c * 64, h, j * 128, b);
+      }
+    }
+    int issued = 0;
+    bool ok = true;
+    for (int idx = 0; idx < ni; ++idx) {
+      const int st = idx & 1;
+      const int i = i0 + idx;
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.qd_empty[st], ((idx >> 1) & 1) ^ 1, wc));
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.qd_full[st], 2 * Cfg::kTileBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c) {
+          tma_load_4d(sm.q[st] + c * Cfg::kChunkBytes, &tm_q, &sm.qd_full[st], c * 64, h, i * 128, b);
+          tma_load_4d(sm.dO[st] + c * Cfg::kChunkBytes, &tm_do, &sm.qd_full[st], c * 64, h, i * 128, b);
+        }
+      }
+      ++issued;
+      for (int t = lane; t < 128; t += 32) {
+        const int qg = i * 128 + t;
+        const int64_t ridx = static_cast<int64_t>(bh) * N + qg;
+        sm.lse2[st][t] = qg < N ? lse[ridx] * kLog2e : INFINITY;
+        sm.dd[st][t] = qg < N ? dsum[ridx] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.qd_full[st]);
+    }
+    if (!ok && lane == 0) {
+      // unwinding: wait (bounded) for the copies in flight
+      mbar_wait_drain(&sm.kv_full, 0, status);
+      for (int idx = (issued > 2 ? issued - 2 : 0); idx < issued; ++idx)
+        mbar_wait_drain(&sm.qd_full[idx & 1], (idx >> 1) & 1, status);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const WaitCtx wc{&sm.abort_flag, status, 12};
+      constexpr uint32_t idesc_sdp = idesc_bf16(128, 128, 0, 0);  // K-major x K-major
+      constexpr uint32_t idesc_acc = idesc_bf16(128, D, 0, 1);    // TMEM A x MN-major B
+      constexpr uint32_t idesc_dq = idesc_bf16(128, D, 1, 1);     // MN-major A (dS) x MN-major B (K)
+      const uint64_t dk_kmaj = sdesc_sw128(smem_u32(sm.k), 16, 1024);
+      const uint64_t dv_kmaj = sdesc_sw128(smem_u32(sm.v), 16, 1024);
+      const uint64_t dk_mn = sdesc_sw128(smem_u32(sm.k), Cfg::kChunkBytes, 1024);
+      const uint64_t dds = sdesc_sw128(smem_u32(sm.ds), 128 * 128, 1024);
+      const uint32_t tS = tbase + Cfg::kColS, tDP = tbase + Cfg::kColDP;
+      const uint32_t tDV = tbase + Cfg::kColDV, tDK = tbase + Cfg::kColDK;
+      auto kmaj_gemm = [&](uint32_t tD, uint64_t da, uint64_t db) {  // (128 x d) . (128 x d)^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * Cfg::kChunkBytes + (kk % 4) * 32) >> 4;
+          umma_ss(tD, da + off, db + off, idesc_sdp, kk > 0);
+        }
+      };
+      bool ok = mbar_wait(&sm.kv_full, 0, wc);
+      for (int idx = 0; idx < ni && ok; ++idx) {
+        const int st = idx & 1;
+        const uint64_t dq_k = sdesc_sw128(smem_u32(sm.q[st]), 16, 1024);
+        const uint64_t ddo_k = sdesc_sw128(smem_u32(sm.dO[st]), 16, 1024);
+        const uint64_t dq_mn = sdesc_sw128(smem_u32(sm.q[st]), Cfg::kChunkBytes, 1024);
+        const uint64_t ddo_mn = sdesc_sw128(smem_u32(sm.dO[st]), Cfg::kChunkBytes, 1024);
+        if (idx == 0) {
+          ok = mbar_wait(&sm.qd_full[0], 0, wc);
+          if (!ok) break;
+          tc_fence_after();
+          kmaj_gemm(tS, dk_kmaj, dq_k);  // S^T = K Q^T
+          umma_commit(&sm.s_full);
+        } else {
+          ok = mbar_wait(&sm.dq_free, (idx - 1) & 1, wc);  // dQ_{i-1} read out of the dP columns
+          if (!ok) break;
+          tc_fence_after();
+        }
+        kmaj_gemm(tDP, dv_kmaj, ddo_k);  // dP^T = V dO^T
+        umma_commit(&sm.dp_full);
+        ok = mbar_wait(&sm.ds_ready, idx & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO   (K = 128 queries)
+          umma_ts(tDV, tS + kk * 8, ddo_mn + ((kk * 2048) >> 4), idesc_acc, (kk > 0) || (idx > 0));
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q
+          umma_ts(tDK, tDP + kk * 8, dq_mn + ((kk * 2048) >> 4), idesc_acc, (kk > 0) || (idx > 0));
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // dQ = dS K   (K = 128 keys) into the dP columns
+          umma_ss(tDP, dds + ((kk * 2048) >> 4), dk_mn + ((kk * 2048) >> 4), idesc_dq, kk > 0);
+        }
+        umma_commit(&sm.dq_full);
+        umma_commit(&sm.qd_empty[st]);
+        if (idx + 1 < ni) {
+          ok = mbar_wait(&sm.qd_full[st ^ 1], ((idx + 1) >> 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dq_k1 = sdesc_sw128(smem_u32(sm.q[st ^ 1]), 16, 1024);
+          kmaj_gemm(tS, dk_kmaj, dq_k1);  // S^T for the next query block
+          umma_commit(&sm.s_full);
+        }
+      }
+      umma_commit(&sm.acc_done);
+      umma_commit(&sm.mma_drain);
+      mbar_wait_drain(&sm.mma_drain, 0, status);
+    }
+    __syncwarp();
+  }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ key rows: P^T, dS^T
+    regs_set<kLaunchRegs, kBwdRegsKey>();
+    const int r = threadIdx.x;  // key row within the block == TMEM lane
+    const int kg = j * 128 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tbase + Cfg::kColS + lane_off;
+    const uint32_t tDP = tbase + Cfg::kColDP + lane_off;
+    const float sl = scale * kLog2e;
+    const WaitCtx wc{&sm.abort_flag, status, 13};
+    uint8_t* ds_row = sm.ds + (r >> 3) * 1024 + (r & 7) * 128;
+    bool ok = true;
+    for (int idx = 0; idx < ni && ok; ++idx) {
+      const int st = idx & 1;
+      const int i = i0 + idx;
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.qd_full[st], (idx >> 1) & 1, wc));
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.s_full, idx & 1, wc));
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.dp_full, idx & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      // valid (query q, key k): k < N, and k <= q when causal; q >= N has LSE = +inf -> P = 0
+      const bool key_ok = kg < N;
+      const int qlim = (CAUSAL && i == j) ? r : 0;  // on the diagonal block: query index >= r
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], dpv[32];
+        tmem_ld32(tS + c * 32, sv);
+        tmem_ld32(tDP + c * 32, dpv);
+        tmem_wait_ld();
+        uint32_t pk[16], dsk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const int ql = c * 32 + x;
+          float p0 = ex2_approx(fmaf(__uint_as_float(sv[x]), sl, -sm.lse2[st][ql]));
+          float p1 = ex2_approx(fmaf(__uint_as_float(sv[x + 1]), sl, -sm.lse2[st][ql + 1]));
+          if (!key_ok || ql < qlim) p0 = 0.f;
+          if (!key_ok || ql + 1 < qlim) p1 = 0.f;
+          const float ds0 = p0 * (__uint_as_float(dpv[x]) - sm.dd[st][ql]);
+          const float ds1 = p1 * (__uint_as_float(dpv[x + 1]) - sm.dd[st][ql + 1]);
+          pk[x / 2] = pack_bf16x2(p0, p1);
+          dsk[x / 2] = pack_bf16x2(ds0, ds1);
+        }
+        tmem_st16(tS + c * 16, pk);
+        tmem_st16(tDP + c * 16, dsk);
+        // dS into shared memory: row r of the 128-byte-swizzled MN-major layout, queries
+        // 32c..32c+31 = four 16-byte units of 64-query chunk c/2
+        uint8_t* base = ds_row + (c >> 1) * 16384;
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int u = ((c & 1) * 4 + y) ^ (r & 7);
+          *reinterpret_cast<uint4*>(base + u * 16) =
+              make_uint4(dsk[4 * y], dsk[4 * y + 1], dsk[4 * y + 2], dsk[4 * y + 3]);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm.ds_ready);
+    }
+    // final dK_j, dV_j rows
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_done, 0, wc));
+    if (ok) {
+      tc_fence_after();
+      const uint32_t tDV = tbase + Cfg::kColDV + lane_off;
+      const uint32_t tDK = tbase + Cfg::kColDK + lane_off;
+      const int64_t orow = ((static_cast<int64_t>(b) * N + kg) * H + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t a[32], g[32];
+        tmem_ld32(tDV + c, a);
+        tmem_ld32(tDK + c, g);
+        tmem_wait_ld();
+        if (kg < N) {
+          uint4* pv = reinterpret_cast<uint4*>(dv + orow + c);
+          uint4* pk = reinterpret_cast<uint4*>(dk + orow + c);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            pv[x] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * x]), __uint_as_float(a[8 * x + 1])),
+                               pack_bf16x2(__uint_as_float(a[8 * x + 2]), __uint_as_float(a[8 * x + 3])),
+                               pack_bf16x2(__uint_as_float(a[8 * x + 4]), __uint_as_float(a[8 * x + 5])),
+                               pack_bf16x2(__uint_as_float(a[8 * x + 6]), __uint_as_float(a[8 * x + 7])));
+            pk[x] = make_uint4(
+                pack_bf16x2(__uint_as_float(g[8 * x]) * scale, __uint_as_float(g[8 * x + 1]) * scale),
+                pack_bf16x2(__uint_as_float(g[8 * x + 2]) * scale, __uint_as_float(g[8 * x + 3]) * scale),
+                pack_bf16x2(__uint_as_float(g[8 * x + 4]) * scale, __uint_as_float(g[8 * x + 5]) * scale),
+                pack_bf16x2(__uint_as_float(g[8 * x + 6]) * scale, __uint_as_float(g[8 * x + 7]) * scale));
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  } else {
+    // ------------------------------------------------------------ dQ drain (warps 4-7)
+    regs_set<kLaunchRegs, kBwdRegsDrain>();
+    const int r = threadIdx.x - 128;  // query row within the block == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tQ = tbase + Cfg::kColDP + lane_off;
+    const WaitCtx wc{&sm.abort_flag, status, 14};
+    for (int idx = 0; idx < ni; ++idx) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, idx & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      const int qg = (i0 + idx) * 128 + r;
+      float* dst = dq_acc + (static_cast<int64_t>(bh) * N + qg) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t a[32];
+        tmem_ld32(tQ + c, a);
+        tmem_wait_ld();
+        if (qg < N) {
+#pragma unroll
+          for (int x = 0; x < 32; x += 4)
+            red_add_v4(dst + c + x, __uint_as_float(a[x]), __uint_as_float(a[x + 1]), __uint_as_float(a[x + 2]),
+                       __uint_as_float(a[x + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.dq_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace fa

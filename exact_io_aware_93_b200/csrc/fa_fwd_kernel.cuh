@@ -16,8 +16,8 @@
 //              in tensor memory; allocates / frees the 512 TMEM columns
 //   warps 10-11 idle
 // Registers: launched at 168 per thread (384 x 168 = 64512); the softmax warpgroups
-// raise theirs to 200 and the producer/MMA warpgroup drops to 96:
-// 2 x 128 x 200 + 128 x 96 = 63488 <= 64512.
+// raise theirs to 200 and the producer/MMA warpgroup drops to 104:
+// 2 x 128 x 200 + 128 x 104 = 64512.
 //
 // Tensor memory (512 columns x 128 lanes of 32 bit):
 //   [0,128)   S_0  (fp32 scores of block 0; P_0 overwrites its first 64 columns as bf16)
@@ -51,9 +51,10 @@ namespace fa {
 constexpr int kBM = 128;  // query rows per block
 constexpr int kBN = 128;  // keys per K/V tile
 constexpr int kFwdThreads = 384;
+constexpr uint32_t kLaunchRegs = 168;  // 65536 / 384 rounded down to a multiple of 8
 constexpr uint32_t kFwdRegsSoftmax = 200;
-constexpr uint32_t kFwdRegsOther = 96;
-static_assert(2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsOther <= kFwdThreads * 168,
+constexpr uint32_t kFwdRegsOther = 104;
+static_assert(2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsOther <= kFwdThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr float kTau = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
@@ -126,6 +127,41 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   return true;
 }
 
+// Which of the 64 column pairs of an unmasked score row take the FMA-pipe exp2
+// (bit c % 8 of the mask): the MUFU unit alone cannot keep pace with the tensor core.
+#ifndef FA_FWD_EMU_MASK
+#define FA_FWD_EMU_MASK 0x00u
+#endif
+
+// Probabilities of one 128-key score row: p = 2^(s * scale_log2 - m), packed to bf16
+// pairs in p[]; adds the fp32 sum to *l and the sum of the bf16-rounded values to *lr.
+template <bool EMU>
+__device__ __forceinline__ void softmax_row(const uint32_t (&s)[kBN], uint32_t (&p)[kBN / 2], float scale_log2,
+                                            float m, float& l, float& lr) {
+  const float2 sl2 = make_float2(scale_log2, scale_log2);
+  const float2 nm2 = make_float2(-m, -m);
+  float2 se[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 sr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < kBN / 2; ++c) {
+    const float2 x = ffma2(make_float2(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sl2, nm2);
+    float2 e;
+    if (EMU && ((FA_FWD_EMU_MASK >> (c & 7)) & 1u)) {
+      e = exp2_poly2(x);
+    } else {
+      e.x = ex2_approx(x.x);
+      e.y = ex2_approx(x.y);
+    }
+    p[c] = pack_bf16x2(e.x, e.y);
+    se[c & 1] = fadd2(se[c & 1], e);
+    // the bf16 weights the P.V product actually uses: O = O_acc / lr is an exact
+    // convex combination of value rows (the rounding of a dominant weight cancels)
+    sr[c & 1] = fadd2(sr[c & 1], make_float2(__uint_as_float(p[c] << 16), __uint_as_float(p[c] & 0xffff0000u)));
+  }
+  l += (se[0].x + se[0].y) + (se[1].x + se[1].y);
+  lr += (sr[0].x + sr[0].y) + (sr[1].x + sr[1].y);
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -173,7 +209,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
 
-  if (warp >= 8) regs_decrease<kFwdRegsOther>();
+  // Each warpgroup's setmaxnreg sits at the top of the branch holding all of that
+  // warpgroup's code, so every instruction after it is compiled within the new limit.
+  if (warp >= 8) {
+    regs_set<kLaunchRegs, kFwdRegsOther>();
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -227,24 +266,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       uint32_t it = 0, qcnt[2] = {0, 0}, pcnt[2] = {0, 0};
       bool ok = true;
 
+      // Descriptors differ only in the start-address field (low 14 bits, 16-byte units),
+      // so each MMA adds an offset to one base descriptor.
+      const uint64_t dq[2] = {sdesc_sw128(q_addr[0], 16, 1024), sdesc_sw128(q_addr[1], 16, 1024)};
+      const uint64_t dk0 = sdesc_sw128(kv_addr0, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(kv_addr0, Cfg::kChunkBytes, 1024);
       auto issue_s = [&](int i, int slot) {
         const uint32_t tS = tbase + i * 128;
-        const uint32_t kaddr = kv_addr0 + slot * Cfg::kTileBytes;
+        const uint64_t dk = dk0 + static_cast<uint64_t>((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * Cfg::kChunkBytes + (kk % 4) * 32;
-          umma_ss(tS, sdesc_sw128(q_addr[i] + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024), idesc_s,
-                  kk > 0);
+          const uint32_t off = ((kk / 4) * Cfg::kChunkBytes + (kk % 4) * 32) >> 4;
+          umma_ss(tS, dq[i] + off, dk + off, idesc_s, kk > 0);
         }
       };
       auto issue_pv = [&](int i, int slot, uint32_t acc) {
         const uint32_t tO = tbase + Cfg::kOCol + i * D;
         const uint32_t tP = tbase + i * 128;
-        const uint32_t vaddr = kv_addr0 + slot * Cfg::kTileBytes;
+        const uint64_t dv = dv0 + static_cast<uint64_t>((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(tO, tP + kk * 8, sdesc_sw128(vaddr + kk * 16 * 128, Cfg::kChunkBytes, 1024), idesc_o,
-                  (kk > 0) || acc);
+          umma_ts(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_o, (kk > 0) || acc);
       };
 
       for (int k = 0; ok; ++k) {
@@ -307,9 +349,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_wait_drain(&sm.mma_drain, 0, status);
     }
     __syncwarp();
-  } else if (warp < 8) {
+  }
+  } else {
     // ------------------------------------------------------------ softmax groups
-    regs_increase<kFwdRegsSoftmax>();
+    regs_set<kLaunchRegs, kFwdRegsSoftmax>();
     const int g = warp >> 2;             // which query block of the pair
     const int r = threadIdx.x & 127;     // row within the block == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -341,7 +384,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tmem_ld32(tS + 96, s + 96);
         tmem_wait_ld();
         const int k0 = j * kBN;
-        if (j == n - 1 && (CAUSAL || (N % kBN) != 0)) {
+        const bool masked = (j == n - 1) && (CAUSAL || (N % kBN) != 0);
+        if (masked) {
           int lim = N - 1 - k0;                    // last valid key column of this tile
           if (CAUSAL) lim = min(lim, row - k0);    // diagonal tile: key <= query
 #pragma unroll
@@ -382,25 +426,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_wait_st();
           }
         }
-        const float2 sl2 = make_float2(scale_log2, scale_log2);
-        const float2 nm2 = make_float2(-m_ref, -m_ref);
         uint32_t p[kBN / 2];
-        float2 se[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        float2 sr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int c = 0; c < kBN / 2; ++c) {
-          const float2 x = ffma2(make_float2(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sl2, nm2);
-          const float p0 = ex2_approx(x.x);
-          const float p1 = ex2_approx(x.y);
-          p[c] = pack_bf16x2(p0, p1);
-          se[c & 1] = fadd2(se[c & 1], make_float2(p0, p1));
-          // the bf16 weights the P.V product actually uses: O = O_acc / lr is an exact
-          // convex combination of value rows (the rounding of a dominant weight cancels)
-          sr[c & 1] = fadd2(sr[c & 1], make_float2(__uint_as_float(p[c] << 16),
-                                                   __uint_as_float(p[c] & 0xffff0000u)));
-        }
-        l += (se[0].x + se[0].y) + (se[1].x + se[1].y);
-        lr += (sr[0].x + sr[0].y) + (sr[1].x + sr[1].y);
+        // masked tiles hold -inf scores: they stay on the MUFU path (2^-inf = 0 exactly)
+        if (masked)
+          softmax_row<false>(s, p, scale_log2, m_ref, l, lr);
+        else
+          softmax_row<true>(s, p, scale_log2, m_ref, l, lr);
         tmem_st32(tS + 0, p);
         tmem_st32(tS + 32, p + 32);
         tmem_wait_st();

@@ -75,6 +75,31 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  float scale, int causal, void* stream);
 
 /*
+ * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ accumulator
+ * [B, H, N, d] followed by the fp32 row sums D_i = sum_x dO_ix O_ix [B, H, N], i.e.
+ * 4*B*H*N*(d+1).  Returns 0 for invalid sizes (B, H, N < 1 or d not 64 / 128).
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass of L = sum(o * dO): dq, dk, dv, recomputing the score tiles from
+ * q, k and the saved lse (no N x N matrix is stored or read).
+ *   q, k, v, o, dO : in,  bf16 [B, N, H, d]   (o and lse as returned by fa_fwd)
+ *   lse            : in,  fp32 [B, H, N]
+ *   dq, dk, dv     : out, bf16 [B, N, H, d]
+ *   workspace      : device scratch of at least fa_bwd_workspace_size(B, H, N, d)
+ *                    bytes, 16-byte aligned, caller-owned; its contents on entry do
+ *                    not matter and are overwritten.
+ *   scale, causal  : the values passed to fa_fwd.
+ * Errors: FA_ERR_WORKSPACE if workspace is NULL or too small; otherwise as fa_fwd.
+ * dk and dv are deterministic; dq is accumulated with fp32 atomics and may differ in
+ * the last bits between runs.  Calls sharing one workspace must not overlap.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                 float scale, int causal, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of the
  * current device: FA_OK, or FA_ERR_TIMEOUT if a kernel gave up a bounded wait
  * since the last call.  Returns FA_ERR_DEVICE if the stream or device reports a

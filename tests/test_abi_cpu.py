@@ -81,3 +81,27 @@ def test_fwd_without_gpu_reports_device(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is visible: the device check passes")
     assert _fwd(lib) == 4
+
+
+def test_bwd_validation_codes(lib):
+    vp = ctypes.c_void_p
+    lib.fa_bwd.argtypes = [vp] * 10 + [ctypes.c_size_t] + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int, vp]
+    lib.fa_bwd.restype = ctypes.c_int
+    lib.fa_bwd_workspace_size.argtypes = [ctypes.c_int] * 4
+    lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
+    ws = lib.fa_bwd_workspace_size(1, 1, 16, 64)
+    assert ws == 16 * 65 * 4
+    assert lib.fa_bwd_workspace_size(1, 1, 16, 96) == 0
+
+    def call(p=0x10000, wsp=0x10000, wsb=ws, d=64, B=1, scale=0.125):
+        return lib.fa_bwd(vp(p), vp(0x10000), vp(0x10000), vp(0x10000), vp(0x10000), vp(0x10000),
+                          vp(0x10000), vp(0x10000), vp(0x10000), vp(wsp), wsb, B, 1, 16, d,
+                          ctypes.c_float(scale), 0, None)
+    assert call(p=0) == 1
+    assert call(B=0) == 1
+    assert call(scale=-1.0) == 1
+    assert call(d=80) == 2
+    assert call(p=0x10001) == 3
+    assert call(wsp=0) == 7
+    assert call(wsb=ws - 1) == 7
+    assert call(wsp=0x10004) == 3
