@@ -62,9 +62,9 @@ def _dist_env():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """nvidia-smi clock / throttle-reason samples, kept only when taken inside the timed region."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -72,15 +72,24 @@ class ClockSampler:
         self.dev = device_index
         self.proc = None
         self.path = os.path.join("/tmp", f"fa_bench_clocks_{os.getpid()}.csv")
+        self.window = None
 
     def start(self):
+        """Start sampling; returns once the first sample has arrived (or after 3 s)."""
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}", "--format=csv,noheader",
-                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
+
+    def mark(self, t_begin: float, t_end: float):
+        self.window = (t_begin, t_end)
 
     def stop(self):
         if self.proc is None:
@@ -91,25 +100,30 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
-        sm, smax, reasons, power = [], [], set(), []
+        import datetime
+        sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1].split()[0]))
-                    smax.append(float(parts[2].split()[0]))
-                    power.append(float(parts[3].split()[0]))
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    clk, cmax = float(parts[2].split()[0]), float(parts[3].split()[0])
+                    pw = float(parts[4].split()[0])
                 except ValueError:
                     continue
-                for name, val in zip(names, parts[5:9]):
+                if self.window and not (self.window[0] - 0.05 <= ts <= self.window[1] + 0.05):
+                    continue
+                sm.append(clk)
+                smax.append(cmax)
+                power.append(pw)
+                for name, val in zip(names, parts[6:10]):
                     if val.lower() == "active":
                         reasons.add(name)
         os.unlink(self.path)
-        loaded = [s for s in sm if smax and s > 0.5 * max(smax)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+        return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "power_w_max": max(power) if power else None,
                 "samples": len(sm), "reasons": sorted(reasons)}
@@ -136,18 +150,27 @@ def _step_fn(api, t, w, with_bwd, events=None):
     return step
 
 
-def cpu_sample(w, heads: int, threads: int):
-    """Time the fp64 oracle on `heads` full heads of workload w (forward and backward)."""
+def cpu_sample(w, heads: int, threads: int, rows: int | None = None, backward: bool = True):
+    """Time the fp64 oracle on `heads` heads of workload w.
+
+    rows=None: every query row of each head; otherwise the forward of the last `rows` query
+    rows (the rows that see the most keys).  backward=True adds the full-head backward.
+    Returns (FLOPs under the benchmark's convention, seconds).
+    """
     import oracle
     oracle.oracle_threads(threads)
-    inp = make_inputs(1, heads, w.N, w.d, w.seed, with_do=with_bwd_available())
+    inp = make_inputs(1, heads, w.N, w.d, w.seed, with_do=backward)
+    sel = None if rows is None else list(range(w.N - rows, w.N))
     t0 = time.perf_counter()
     flops = 0.0
     for h in range(heads):
         q, k, v = (inp[n][0, :, h].double().numpy() for n in ("q", "k", "v"))
-        oracle.fwd_rows(q, k, v, w.scale, w.causal)
-        flops += fwd_flops(1, 1, w.N, w.d, w.causal)
-        if with_bwd_available():
+        oracle.fwd_rows(q, k, v, w.scale, w.causal, sel)
+        if sel is None:
+            flops += fwd_flops(1, 1, w.N, w.d, w.causal)
+        else:
+            flops += sum(4.0 * ((i + 1) if w.causal else w.N) * w.d for i in sel)
+        if backward:
             do = inp["do"][0, :, h].double().numpy()
             oracle.bwd_rows(q, k, v, do, w.scale, w.causal)
             flops += bwd_flops(1, 1, w.N, w.d, w.causal)
@@ -163,22 +186,41 @@ def with_bwd_available() -> bool:
         return False
 
 
+REFERENCE_BUDGET_S = 150.0
+
+
 def run_reference(args, w):
+    """The fp64 oracle on the host cores, each step a sample of the same workload sized so the
+    whole run (warm-up + timed steps) stays within about REFERENCE_BUDGET_S seconds."""
     world, rank, _ = _dist_env()
     if rank != 0:
         return 0
     threads = len(os.sched_getaffinity(0))
-    heads = 1
+    per_step = REFERENCE_BUDGET_S / (args.warmup + args.steps)
+    # calibrate the oracle's rate on a small forward sample
+    cf, ct = cpu_sample(w, 1, threads, rows=256, backward=False)
+    rate = cf / ct
+    full = fwd_flops(1, 1, w.N, w.d, w.causal) + (bwd_flops(1, 1, w.N, w.d, w.causal) if w.backward else 0.0)
+    if full / rate <= per_step:
+        kw = {"rows": None, "backward": w.backward}
+        sample = f"1 full head (b=0, h=0) of {w.name}: forward" + (" and backward" if w.backward else "") \
+                 + " of every row, fp64"
+    else:
+        rows = w.N
+        while rows > 64 and sum(4.0 * ((i + 1) if w.causal else w.N) * w.d
+                                for i in range(w.N - rows, w.N)) / rate > per_step:
+            rows //= 2
+        kw = {"rows": None if rows == w.N else rows, "backward": False}
+        sample = (f"forward of the last {rows} query rows of head (b=0, h=0) of {w.name}, fp64 "
+                  f"(backward left out so {args.warmup + args.steps} steps fit ~{REFERENCE_BUDGET_S:.0f} s)")
     times = []
     flops_step = 0.0
     for i in range(args.warmup + args.steps):
-        flops_step, dt = cpu_sample(w, heads, threads)
+        flops_step, dt = cpu_sample(w, 1, threads, **kw)
         if i >= args.warmup:
             times.append(dt)
     total = sum(times)
     value = flops_step * len(times) / total / 1e12
-    sample = (f"{heads} full head(s) (b=0, h=0) of {w.name}: forward"
-              + (" and backward" if with_bwd_available() else "") + " of every row, fp64")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -214,6 +256,8 @@ def run_ours(args, w):
     in_bytes = sum(t[n].numel() * t[n].element_size() for n in ("q", "k", "v", "do"))
 
     step = _step_fn(api, t, w, with_bwd)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -223,20 +267,21 @@ def run_ours(args, w):
     # ---------------- device-timed region
     events = {"fwd": [], "bwd": []}
     tstep = _step_fn(api, t, w, with_bwd, events)
-    clocks = ClockSampler(dev.index)
-    clocks.start()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_begin = time.time()
     e0.record()
     for _ in range(args.steps):
         tstep()
     e1.record()
     torch.cuda.synchronize()
+    t_end = time.time()
     if world > 1:
         dist.barrier()
+    clocks.mark(t_begin, t_end)
     clk = clocks.stop()
     ms = e0.elapsed_time(e1) / args.steps
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in events["fwd"])
@@ -313,7 +358,7 @@ def run_ours(args, w):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = len(os.sched_getaffinity(0))
         heads = 4
-        cflops, cdt = cpu_sample(w, heads, threads)
+        cflops, cdt = cpu_sample(w, heads, threads, backward=with_bwd)
         line["cpu_baseline"] = {
             "value": cflops / cdt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
             "sample": f"{heads} full heads of {w.name} (forward" + (" + backward" if with_bwd else "")
@@ -329,8 +374,8 @@ def run_ours(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
