@@ -5,6 +5,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/fa.h"
 #include "fa_bwd_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
@@ -146,6 +148,43 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   return FA_OK;
 }
 
+// ---------------------------------------------------------------- allocation-free backward
+// Scratch for fa_bwd_noalloc: a fixed device array in this module, so callers that may not
+// allocate device memory still get a backward pass.  It exists on every GPU that loads the
+// library, for the life of the process, and every fa_bwd_noalloc call on a device uses it.
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(64) << 20;  // 64 MiB
+static __device__ __align__(256) uint8_t g_fa_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocScratch {
+  bool ready = false;
+  void* ptr = nullptr;  // device address of g_fa_noalloc_scratch on this device
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+std::mutex g_noalloc_mutex;
+
+// Per-device set-up, done once with the device current: in host code the array's name is
+// only a stand-in, so the kernels get the address the runtime reports for this device.
+fa_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  NoAllocScratch& ns = g_noalloc[dev];
+  if (!ns.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return FA_ERR_DEVICE;
+    }
+    ns.ptr = p;
+    ns.ready = true;
+  }
+  *out = ns.ptr;
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -218,6 +257,19 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                   : launch_bwd<128, false>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s);
   return causal ? launch_bwd<64, true>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s)
                 : launch_bwd<64, false>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s);
+}
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                         int causal, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  const fa_status st = check_common(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (bwd_ws_bytes(B, H, N, d) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const fa_status ss = noalloc_scratch(&scratch);
+  if (ss != FA_OK) return ss;
+  return fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, scratch, kNoAllocScratchBytes, B, H, N, d, scale, causal, stream);
 }
 
 fa_status fa_get_status(void* stream) {

@@ -100,6 +100,29 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  float scale, int causal, void* stream);
 
 /*
+ * fa_bwd without a workspace argument, for callers that cannot allocate device memory:
+ * for example code running where every byte of device memory is already handed to
+ * another allocator, or where the implicit synchronisation of cudaMalloc / cudaFree is
+ * not acceptable.  (The pages describe no such entry point; it has no counterpart there.)
+ * It performs the same computation as fa_bwd, with the same arguments minus the
+ * workspace, and calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Scratch: a fixed 64 MiB array inside the library (fp32 dQ accumulator and row sums,
+ * 4*B*H*N*(d+1) bytes).  Problems that need more return FA_ERR_WORKSPACE and launch
+ * nothing; use fa_bwd with a caller-provided workspace for those.  Every GPU that loads
+ * the library holds this array until the process exits, whether or not this entry point
+ * is used.  All calls on a device share the one array: calls whose work can overlap on
+ * the GPU (different streams without ordering between them) race and corrupt each
+ * other's results; serialise them.  Whatever must start at zero is cleared by each call.
+ *
+ * The first call on each device looks up the array's device address (once per device,
+ * with that device current); make that first call before any CUDA stream capture.
+ */
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                         int causal, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of the
  * current device: FA_OK, or FA_ERR_TIMEOUT if a kernel gave up a bounded wait
  * since the last call.  Returns FA_ERR_DEVICE if the stream or device reports a
