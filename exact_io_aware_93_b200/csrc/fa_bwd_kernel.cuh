@@ -18,14 +18,20 @@
 //                   dS^T = P^T o (dP^T - D_i)
 //                   dV_j += P^T dO_i        (A operand P^T read from tensor memory)
 //                   dK_j += dS^T Q_i        (A operand dS^T read from tensor memory)
-//                   dQ_i  = dS K_j          (dS written to shared memory, 128-byte swizzle)
-//                 and a drain warpgroup adds each dQ_i tile into the fp32 accumulator with
-//                 vector reductions; dK_j, dV_j are written once at the end.
+//                   dQ_i  = dS K_j          (dS written to shared memory, 128-byte swizzle);
+//                                           for d = 128 computed transposed, dQ_i^T = K_j^T dS^T,
+//                                           so that tensor-memory lanes are head-dim columns
+//                 and a drain warpgroup copies each dQ_i tile out of tensor memory, frees it,
+//                 and adds it into the fp32 accumulator with reductions that cover whole
+//                 128-byte lines; dK_j, dV_j are written once at the end.
+//   Per query block the MMA warp issues dP, then (once P is ready) dV and the next block's
+//   S, then (once dS is ready) dK and dQ, so the tensor core works while the key-row
+//   warpgroup computes dS and while the drain empties the previous dQ tile.
 //   fa_bwd_post : dQ = bf16(scale * accumulator)
 //
 // Tensor memory (512 columns):
 //   [0,128)   S^T  (fp32; P^T overwrites its first 64 columns as bf16)
-//   [128,256) dP^T (fp32; dS^T overwrites its first 64 columns; then dQ_i, fp32, D columns)
+//   [128,256) dP^T (fp32; dS^T overwrites its first 64 columns; then dQ_i (or dQ_i^T), fp32)
 //   [256,256+D) dV_j accumulator,  [384,384+D) dK_j accumulator
 //
 // Warp roles (384 threads): warps 0-3 key rows (P, dS, final dK/dV), warps 4-7 dQ drain,
@@ -39,7 +45,7 @@ namespace fa {
 
 constexpr int kBwdThreads = 384;
 constexpr uint32_t kBwdRegsKey = 224;
-constexpr uint32_t kBwdRegsDrain = 128;
+constexpr uint32_t kBwdRegsDrain = 160;
 constexpr uint32_t kBwdRegsOther = 96;
 static_assert(128 * (kBwdRegsKey + kBwdRegsDrain + kBwdRegsOther) <= kBwdThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
@@ -70,6 +76,7 @@ struct __align__(1024) BwdSmem {
   uint64_t qd_empty[2];
   uint64_t s_full;
   uint64_t dp_full;
+  uint64_t p_ready;
   uint64_t ds_ready;
   uint64_t dq_full;
   uint64_t dq_free;
@@ -141,6 +148,10 @@ __global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restric
   *reinterpret_cast<uint4*>(dq + ((static_cast<int64_t>(b) * N + n) * H + h) * D + part * 8) = r;
 }
 
+__device__ __forceinline__ void red_add(float* addr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
+}
+
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
@@ -181,6 +192,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(&sm.s_full, 1);
     mbar_init(&sm.dp_full, 1);
+    mbar_init(&sm.p_ready, 128);
     mbar_init(&sm.ds_ready, 128);
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_free, 128);
@@ -265,51 +277,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           umma_ss(tD, da + off, db + off, idesc_sdp, kk > 0);
         }
       };
-      bool ok = mbar_wait(&sm.kv_full, 0, wc);
+      constexpr bool kDqT = (D == 128);  // dQ^T = K^T dS^T: M = d, N = 128 queries
+      constexpr uint32_t idesc_dqt = idesc_bf16(128, 128, 1, 1);
+      bool ok = mbar_wait(&sm.kv_full, 0, wc) && mbar_wait(&sm.qd_full[0], 0, wc);
+      if (ok) {
+        tc_fence_after();
+        kmaj_gemm(tS, dk_kmaj, sdesc_sw128(smem_u32(sm.q[0]), 16, 1024));  // S^T for the first block
+        umma_commit(&sm.s_full);
+      }
       for (int idx = 0; idx < ni && ok; ++idx) {
         const int st = idx & 1;
-        const uint64_t dq_k = sdesc_sw128(smem_u32(sm.q[st]), 16, 1024);
         const uint64_t ddo_k = sdesc_sw128(smem_u32(sm.dO[st]), 16, 1024);
         const uint64_t dq_mn = sdesc_sw128(smem_u32(sm.q[st]), Cfg::kChunkBytes, 1024);
         const uint64_t ddo_mn = sdesc_sw128(smem_u32(sm.dO[st]), Cfg::kChunkBytes, 1024);
-        if (idx == 0) {
-          ok = mbar_wait(&sm.qd_full[0], 0, wc);
-          if (!ok) break;
-          tc_fence_after();
-          kmaj_gemm(tS, dk_kmaj, dq_k);  // S^T = K Q^T
-          umma_commit(&sm.s_full);
-        } else {
-          ok = mbar_wait(&sm.dq_free, (idx - 1) & 1, wc);  // dQ_{i-1} read out of the dP columns
+        if (idx > 0) {
+          ok = mbar_wait(&sm.dq_free, (idx - 1) & 1, wc);  // dQ_{i-1} copied out of the dP columns
           if (!ok) break;
           tc_fence_after();
         }
         kmaj_gemm(tDP, dv_kmaj, ddo_k);  // dP^T = V dO^T
         umma_commit(&sm.dp_full);
-        ok = mbar_wait(&sm.ds_ready, idx & 1, wc);
+        ok = mbar_wait(&sm.p_ready, idx & 1, wc);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO   (K = 128 queries)
           umma_ts(tDV, tS + kk * 8, ddo_mn + ((kk * 2048) >> 4), idesc_acc, (kk > 0) || (idx > 0));
         }
+        if (idx + 1 < ni) {  // next block's S^T, into the columns P^T just left
+          ok = mbar_wait(&sm.qd_full[st ^ 1], ((idx + 1) >> 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          kmaj_gemm(tS, dk_kmaj, sdesc_sw128(smem_u32(sm.q[st ^ 1]), 16, 1024));
+          umma_commit(&sm.s_full);
+        }
+        ok = mbar_wait(&sm.ds_ready, idx & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q
           umma_ts(tDK, tDP + kk * 8, dq_mn + ((kk * 2048) >> 4), idesc_acc, (kk > 0) || (idx > 0));
         }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // dQ = dS K   (K = 128 keys) into the dP columns
-          umma_ss(tDP, dds + ((kk * 2048) >> 4), dk_mn + ((kk * 2048) >> 4), idesc_dq, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) {  // dQ (K = 128 keys) into the dP columns
+          if constexpr (kDqT)
+            umma_ss(tDP, dk_mn + ((kk * 2048) >> 4), dds + ((kk * 2048) >> 4), idesc_dqt, kk > 0);
+          else
+            umma_ss(tDP, dds + ((kk * 2048) >> 4), dk_mn + ((kk * 2048) >> 4), idesc_dq, kk > 0);
         }
         umma_commit(&sm.dq_full);
         umma_commit(&sm.qd_empty[st]);
-        if (idx + 1 < ni) {
-          ok = mbar_wait(&sm.qd_full[st ^ 1], ((idx + 1) >> 1) & 1, wc);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t dq_k1 = sdesc_sw128(smem_u32(sm.q[st ^ 1]), 16, 1024);
-          kmaj_gemm(tS, dk_kmaj, dq_k1);  // S^T for the next query block
-          umma_commit(&sm.s_full);
-        }
       }
       umma_commit(&sm.acc_done);
       umma_commit(&sm.mma_drain);
@@ -328,38 +345,77 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float sl = scale * kLog2e;
     const WaitCtx wc{&sm.abort_flag, status, 13};
     uint8_t* ds_row = sm.ds + (r >> 3) * 1024 + (r & 7) * 128;
+    const float2 sl2 = make_float2(sl, sl);
     bool ok = true;
     for (int idx = 0; idx < ni && ok; ++idx) {
       const int st = idx & 1;
       const int i = i0 + idx;
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.qd_full[st], (idx >> 1) & 1, wc));
       ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.s_full, idx & 1, wc));
-      ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.dp_full, idx & 1, wc));
       if (!ok) break;
       tc_fence_after();
       // valid (query q, key k): k < N, and k <= q when causal; q >= N has LSE = +inf -> P = 0
       const bool key_ok = kg < N;
       const int qlim = (CAUSAL && i == j) ? r : 0;  // on the diagonal block: query index >= r
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32], dpv[32];
-        tmem_ld32(tS + c * 32, sv);
-        tmem_ld32(tDP + c * 32, dpv);
-        tmem_wait_ld();
-        uint32_t pk[16], dsk[16];
+      const bool masked = __any_sync(0xffffffffu, !key_ok || qlim > 0);
+      const float* lse2 = sm.lse2[st];
+      const float* dd = sm.dd[st];
+      float pf[128];  // fp32 P^T of this key row, kept for dS
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32];
+        tmem_ld32(tS + c * 32, sv);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 4) {
           const int ql = c * 32 + x;
-          float p0 = ex2_approx(fmaf(__uint_as_float(sv[x]), sl, -sm.lse2[st][ql]));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sv[x + 1]), sl, -sm.lse2[st][ql + 1]));
-          if (!key_ok || ql < qlim) p0 = 0.f;
-          if (!key_ok || ql + 1 < qlim) p1 = 0.f;
-          const float ds0 = p0 * (__uint_as_float(dpv[x]) - sm.dd[st][ql]);
-          const float ds1 = p1 * (__uint_as_float(dpv[x + 1]) - sm.dd[st][ql + 1]);
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + ql);
+          const float2 a = ffma2(make_float2(__uint_as_float(sv[x]), __uint_as_float(sv[x + 1])), sl2,
+                                 make_float2(-l4.x, -l4.y));
+          const float2 b = ffma2(make_float2(__uint_as_float(sv[x + 2]), __uint_as_float(sv[x + 3])), sl2,
+                                 make_float2(-l4.z, -l4.w));
+          float p0 = ex2_approx(a.x), p1 = ex2_approx(a.y), p2 = ex2_approx(b.x), p3 = ex2_approx(b.y);
+          if (masked) {
+            if (!key_ok || ql < qlim) p0 = 0.f;
+            if (!key_ok || ql + 1 < qlim) p1 = 0.f;
+            if (!key_ok || ql + 2 < qlim) p2 = 0.f;
+            if (!key_ok || ql + 3 < qlim) p3 = 0.f;
+          }
+          pf[ql] = p0;
+          pf[ql + 1] = p1;
+          pf[ql + 2] = p2;
+          pf[ql + 3] = p3;
           pk[x / 2] = pack_bf16x2(p0, p1);
-          dsk[x / 2] = pack_bf16x2(ds0, ds1);
+          pk[x / 2 + 1] = pack_bf16x2(p2, p3);
         }
         tmem_st16(tS + c * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.p_ready);
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.dp_full, idx & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t dpv[32];
+        tmem_ld32(tDP + c * 32, dpv);
+        tmem_wait_ld();
+        uint32_t dsk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 4) {
+          const int ql = c * 32 + x;
+          const float4 d4 = *reinterpret_cast<const float4*>(dd + ql);
+          const float2 a = fmul2(make_float2(pf[ql], pf[ql + 1]),
+                                 fadd2(make_float2(__uint_as_float(dpv[x]), __uint_as_float(dpv[x + 1])),
+                                       make_float2(-d4.x, -d4.y)));
+          const float2 b = fmul2(make_float2(pf[ql + 2], pf[ql + 3]),
+                                 fadd2(make_float2(__uint_as_float(dpv[x + 2]), __uint_as_float(dpv[x + 3])),
+                                       make_float2(-d4.z, -d4.w)));
+          dsk[x / 2] = pack_bf16x2(a.x, a.y);
+          dsk[x / 2 + 1] = pack_bf16x2(b.x, b.y);
+        }
         tmem_st16(tDP + c * 16, dsk);
         // dS into shared memory: row r of the 128-byte-swizzled MN-major layout, queries
         // 32c..32c+31 = four 16-byte units of 64-query chunk c/2
@@ -411,7 +467,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // ------------------------------------------------------------ dQ drain (warps 4-7)
     regs_set<kLaunchRegs, kBwdRegsDrain>();
-    const int r = threadIdx.x - 128;  // query row within the block == TMEM lane
+    const int r = threadIdx.x - 128;  // TMEM lane: head-dim column (d = 128) or query row (d = 64)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tQ = tbase + Cfg::kColDP + lane_off;
     const WaitCtx wc{&sm.abort_flag, status, 14};
@@ -419,22 +475,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, idx & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      const int qg = (i0 + idx) * 128 + r;
-      float* dst = dq_acc + (static_cast<int64_t>(bh) * N + qg) * D;
-#pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t a[32];
-        tmem_ld32(tQ + c, a);
+      const int q0 = (i0 + idx) * 128;
+      if constexpr (D == 128) {
+        // lane r holds column r of dQ_i for the 128 queries; a warp's reduction for one query
+        // covers 32 consecutive columns = one 128-byte line
+        uint32_t a[128];
+        tmem_ld32(tQ + 0, a);
+        tmem_ld32(tQ + 32, a + 32);
+        tmem_ld32(tQ + 64, a + 64);
+        tmem_ld32(tQ + 96, a + 96);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&sm.dq_free);  // the dP columns may be overwritten from here on
+        const int qn = min(128, N - q0);
+        float* dst = dq_acc + (static_cast<int64_t>(bh) * N + q0) * D + r;
+#pragma unroll
+        for (int q = 0; q < 128; ++q)
+          if (q < qn) red_add(dst + static_cast<int64_t>(q) * D, __uint_as_float(a[q]));
+      } else {
+        const int qg = q0 + r;
+        float* dst = dq_acc + (static_cast<int64_t>(bh) * N + qg) * D;
+        uint32_t a[D];
+#pragma unroll
+        for (int c = 0; c < D; c += 32) tmem_ld32(tQ + c, a + c);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&sm.dq_free);
         if (qg < N) {
 #pragma unroll
-          for (int x = 0; x < 32; x += 4)
-            red_add_v4(dst + c + x, __uint_as_float(a[x]), __uint_as_float(a[x + 1]), __uint_as_float(a[x + 2]),
+          for (int x = 0; x < D; x += 4)
+            red_add_v4(dst + x, __uint_as_float(a[x]), __uint_as_float(a[x + 1]), __uint_as_float(a[x + 2]),
                        __uint_as_float(a[x + 3]));
         }
       }
-      tc_fence_before();
-      mbar_arrive(&sm.dq_free);
     }
   }
 
