@@ -35,13 +35,13 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // split is computed for a launch at exactly fa::kLaunchRegs registers per thread.
 // Refuse to launch a build whose register count differs.
 template <typename K>
-bool launch_regs_ok(K kern) {
+bool launch_regs_ok(K kern, uint32_t expected) {
   cudaFuncAttributes a;
   if (cudaFuncGetAttributes(&a, kern) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
-  return a.numRegs == static_cast<int>(fa::kLaunchRegs);
+  return a.numRegs == static_cast<int>(expected);
 }
 
 fa_status current_device(DeviceInfo** out) {
@@ -91,7 +91,7 @@ fa_status launch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   const int smem = static_cast<int>(sizeof(fa::FwdSmem<D>)) + 1024;
   bool& attr = di.fwd_attr[D == 128][CAUSAL];
   if (!attr) {
-    if (!launch_regs_ok(kern) ||
+    if (!launch_regs_ok(kern, fa::kLaunchRegs) ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
       cudaGetLastError();
       return FA_ERR_LAUNCH;
@@ -108,9 +108,12 @@ fa_status launch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   return FA_OK;
 }
 
+// Workspace: fp32 dQ accumulator [B, H, N, d], then fp32 D and fp32 LSE * log2(e), each
+// [B*H, Npad] with Npad = N rounded up to a multiple of 128.
 size_t bwd_ws_bytes(int B, int H, int N, int d) {
-  const size_t rows = static_cast<size_t>(B) * H * N;
-  return rows * static_cast<size_t>(d) * 4 + rows * 4;  // fp32 dQ accumulator + fp32 D
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  return bh * static_cast<size_t>(N) * static_cast<size_t>(d) * 4 + 2 * bh * npad * 4;
 }
 
 template <int D, bool CAUSAL>
@@ -118,19 +121,22 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
                      const CUtensorMap& mdo, const void* o, const void* dO, const float* lse, void* dq, void* dk,
                      void* dv, void* ws, int B, int H, int N, float scale, cudaStream_t stream) {
   const int64_t rows = static_cast<int64_t>(B) * H * N;
+  const int64_t prows = static_cast<int64_t>(B) * H * ((N + 127) / 128 * 128);
   float* dq_acc = static_cast<float*>(ws);
   float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + rows * D * 4);
+  float* lse2 = dsum + prows;
+  const unsigned pre_blocks = static_cast<unsigned>((prows * (D / 8) + 255) / 256);
+  fa::fa_bwd_pre_kernel<D><<<pre_blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                           static_cast<const __nv_bfloat16*>(dO), lse, dsum, lse2,
+                                                           dq_acc, B, H, N);
   const int64_t ew_threads = rows * (D / 8);
   const unsigned ew_blocks = static_cast<unsigned>((ew_threads + 255) / 256);
-  fa::fa_bwd_pre_kernel<D><<<ew_blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                          static_cast<const __nv_bfloat16*>(dO), dsum, dq_acc, B,
-                                                          H, N);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   auto kern = fa::fa_bwd_main_kernel<D, CAUSAL>;
   const int smem = static_cast<int>(sizeof(fa::BwdSmem<D>));
   bool& attr = di.bwd_attr[D == 128][CAUSAL];
   if (!attr) {
-    if (!launch_regs_ok(kern) ||
+    if (!launch_regs_ok(kern, fa::kBwdLaunchRegs) ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
       cudaGetLastError();
       return FA_ERR_LAUNCH;
@@ -138,7 +144,7 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
     attr = true;
   }
   const int nkb = (N + 127) / 128;
-  kern<<<B * H * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, lse, dsum, dq_acc,
+  kern<<<B * H * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, lse2, dsum, dq_acc,
                                                         static_cast<__nv_bfloat16*>(dk),
                                                         static_cast<__nv_bfloat16*>(dv), B, H, N, scale, di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;

@@ -9,13 +9,14 @@
 // D_i equals the Jacobian row constant sum_t P_it dP_it because O_i = sum_t P_it v_t.
 //
 // Three kernels, one stream:
-//   fa_bwd_pre  : D_i (fp32) and zeroing of the fp32 dQ accumulator (memory bound)
+//   fa_bwd_pre  : D_i and LSE_i * log2 e (fp32, padded per head to whole 128-row blocks) and
+//                 zeroing of the fp32 dQ accumulator (memory bound)
 //   fa_bwd_main : one CTA per (batch, head, 128-key block j); K_j and V_j stay in shared
 //                 memory while 128-query blocks i (i >= j when causal) stream through:
 //                   S^T  = K_j Q_i^T        (tcgen05, both operands in shared memory)
 //                   dP^T = V_j dO_i^T
 //                   P^T  = 2^(S^T * scale * log2 e - LSE_i * log2 e)   (one thread per key)
-//                   dS^T = P^T o (dP^T - D_i)
+//                   dS^T = P^T o (dP^T - D_i)   (with the bf16 P^T that enters dV)
 //                   dV_j += P^T dO_i        (A operand P^T read from tensor memory)
 //                   dK_j += dS^T Q_i        (A operand dS^T read from tensor memory)
 //                   dQ_i  = dS K_j          (dS written to shared memory, 128-byte swizzle);
@@ -30,12 +31,15 @@
 //   fa_bwd_post : dQ = bf16(scale * accumulator)
 //
 // Tensor memory (512 columns):
-//   [0,128)   S^T  (fp32; P^T overwrites its first 64 columns as bf16)
-//   [128,256) dP^T (fp32; dS^T overwrites its first 64 columns; then dQ_i (or dQ_i^T), fp32)
+//   [0,128)   S^T  (fp32).  Key-row warpgroup g (queries 64g..64g+63) reads columns
+//             [64g, 64g+64) and writes its bf16 P^T into [64g, 64g+32), inside its own range.
+//   [128,256) dP^T (fp32), dS^T likewise at [128+64g, 128+64g+32); then dQ_i (or dQ_i^T), fp32
 //   [256,256+D) dV_j accumulator,  [384,384+D) dK_j accumulator
 //
-// Warp roles (384 threads): warps 0-3 key rows (P, dS, final dK/dV), warps 4-7 dQ drain,
-// warp 8 loads (TMA for tiles, plain loads for LSE and D), warp 9 issues MMAs.
+// Warp roles (512 threads): warps 0-3 and 4-7 key rows for queries 0-63 and 64-127 of the
+// block (P, dS; at the end dV and dK respectively), warps 8-11 dQ drain, warp 12 loads (TMA
+// tiles for Q, dO and bulk copies of the block's LSE * log2 e and D), warp 13 issues MMAs,
+// warps 14-15 idle.
 #pragma once
 
 #include "fa_fwd_kernel.cuh"
@@ -43,11 +47,12 @@
 
 namespace fa {
 
-constexpr int kBwdThreads = 384;
-constexpr uint32_t kBwdRegsKey = 224;
-constexpr uint32_t kBwdRegsDrain = 160;
+constexpr int kBwdThreads = 512;
+constexpr uint32_t kBwdLaunchRegs = 128;  // 65536 / 512
+constexpr uint32_t kBwdRegsKey = 112;     // two key-row warpgroups
+constexpr uint32_t kBwdRegsDrain = 168;
 constexpr uint32_t kBwdRegsOther = 96;
-static_assert(128 * (kBwdRegsKey + kBwdRegsDrain + kBwdRegsOther) <= kBwdThreads * kLaunchRegs,
+static_assert(128 * (2 * kBwdRegsKey + kBwdRegsDrain + kBwdRegsOther) <= kBwdThreads * kBwdLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -87,21 +92,27 @@ struct __align__(1024) BwdSmem {
 };
 
 // ---------------------------------------------------------------- pre
-// D[b,h,n] = sum_x dO[b,n,h,x] * O[b,n,h,x]; zero the dQ accumulator rows.
-// One group of D/8 threads per row, 16-byte loads.
+// For each (b, h) row n < N: D[bh, n] = sum_x dO[b,n,h,x] * O[b,n,h,x], LSE2[bh, n] =
+// LSE[b,h,n] * log2(e), and the dQ accumulator row set to zero.  D and LSE2 are laid out
+// [B*H, Npad] with Npad = N rounded up to 128; rows n in [N, Npad) get D = 0 and
+// LSE2 = +inf, so every 128-row block is a full, 16-byte-aligned 512-byte run and its
+// padded queries have P = 0.  One group of D/8 threads per row, 16-byte loads.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
-                                                         float* __restrict__ dsum, float* __restrict__ dq_acc,
-                                                         int B, int H, int N) {
+                                                         const float* __restrict__ lse,
+                                                         float* __restrict__ dsum, float* __restrict__ lse2,
+                                                         float* __restrict__ dq_acc, int B, int H, int N) {
   constexpr int TPR = D / 8;  // threads per row
-  const int64_t rows = static_cast<int64_t>(B) * H * N;
+  const int npad = (N + 127) / 128 * 128;
+  const int64_t rows = static_cast<int64_t>(B) * H * npad;
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TPR;
   const int part = threadIdx.x % TPR;
   float acc = 0.f;
-  if (row < rows) {
-    const int64_t bh = row / N;
-    const int n = static_cast<int>(row % N);
+  const int64_t bh = row / npad;
+  const int n = static_cast<int>(row % npad);
+  const bool live = row < rows && n < N;
+  if (live) {
     const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
     const int64_t off = ((static_cast<int64_t>(b) * N + n) * H + h) * D + part * 8;
     const uint4 ov = *reinterpret_cast<const uint4*>(o + off);
@@ -115,13 +126,16 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
       acc = fmaf(a.x, c.x, acc);
       acc = fmaf(a.y, c.y, acc);
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
+    float4* z = reinterpret_cast<float4*>(dq_acc + (bh * N + n) * D + part * 8);
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
   for (int s = TPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (row < rows && part == 0) dsum[row] = acc;
+  if (row < rows && part == 0) {
+    dsum[row] = live ? acc : 0.f;
+    lse2[row] = live ? lse[bh * N + n] * 1.4426950408889634f : INFINITY;
+  }
 }
 
 // ---------------------------------------------------------------- post
@@ -162,7 +176,7 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                       const float* __restrict__ lse, const float* __restrict__ dsum,
+                       const float* __restrict__ lse2g, const float* __restrict__ dsum,
                        float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                        int B, int H, int N, float scale, int* status) {
   using Cfg = BwdCfg<D>;
@@ -187,20 +201,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     sm.abort_flag = 0;
     mbar_init(&sm.kv_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.qd_full[s], 2);  // expect-tx arrive + arrive after LSE / D stores
+      mbar_init(&sm.qd_full[s], 1);
       mbar_init(&sm.qd_empty[s], 1);
     }
     mbar_init(&sm.s_full, 1);
     mbar_init(&sm.dp_full, 1);
-    mbar_init(&sm.p_ready, 128);
-    mbar_init(&sm.ds_ready, 128);
+    mbar_init(&sm.p_ready, 256);
+    mbar_init(&sm.ds_ready, 256);
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_free, 128);
     mbar_init(&sm.acc_done, 1);
     mbar_init(&sm.mma_drain, 1);
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
@@ -211,9 +225,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   // Each warpgroup's setmaxnreg sits at the top of the branch holding all of that
   // warpgroup's code, so every instruction after it is compiled within the new limit.
-  if (warp >= 8) {
-    regs_set<kLaunchRegs, kBwdRegsOther>();
-  if (warp == 8) {
+  if (warp >= 12) {
+    regs_set<kBwdLaunchRegs, kBwdRegsOther>();
+  if (warp == 12) {
     // ------------------------------------------------------------ loads
     const WaitCtx wc{&sm.abort_flag, status, 11};
     if (lane == 0) {
@@ -227,6 +241,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_4d(sm.v + c * Cfg::kChunkBytes, &tm_v, &sm.kv_full, c * 64, h, j * 128, b);
       }
     }
+    const int npad = nkb * 128;
     int issued = 0;
     bool ok = true;
     for (int idx = 0; idx < ni; ++idx) {
@@ -235,21 +250,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.qd_empty[st], ((idx >> 1) & 1) ^ 1, wc));
       if (!ok) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&sm.qd_full[st], 2 * Cfg::kTileBytes);
+        // Q_i, dO_i tiles plus the block's LSE2 and D runs (512 bytes each, padded rows)
+        mbar_arrive_expect_tx(&sm.qd_full[st], 2 * Cfg::kTileBytes + 2 * 512);
         for (int c = 0; c < Cfg::kChunks; ++c) {
           tma_load_4d(sm.q[st] + c * Cfg::kChunkBytes, &tm_q, &sm.qd_full[st], c * 64, h, i * 128, b);
           tma_load_4d(sm.dO[st] + c * Cfg::kChunkBytes, &tm_do, &sm.qd_full[st], c * 64, h, i * 128, b);
         }
+        const int64_t ridx = static_cast<int64_t>(bh) * npad + i * 128;
+        bulk_load(sm.lse2[st], lse2g + ridx, 512, &sm.qd_full[st]);
+        bulk_load(sm.dd[st], dsum + ridx, 512, &sm.qd_full[st]);
       }
       ++issued;
-      for (int t = lane; t < 128; t += 32) {
-        const int qg = i * 128 + t;
-        const int64_t ridx = static_cast<int64_t>(bh) * N + qg;
-        sm.lse2[st][t] = qg < N ? lse[ridx] * kLog2e : INFINITY;
-        sm.dd[st][t] = qg < N ? dsum[ridx] : 0.f;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.qd_full[st]);
     }
     if (!ok && lane == 0) {
       // unwinding: wait (bounded) for the copies in flight
@@ -257,7 +268,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int idx = (issued > 2 ? issued - 2 : 0); idx < issued; ++idx)
         mbar_wait_drain(&sm.qd_full[idx & 1], (idx >> 1) & 1, status);
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const WaitCtx wc{&sm.abort_flag, status, 12};
@@ -302,7 +313,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO   (K = 128 queries)
-          umma_ts(tDV, tS + kk * 8, ddo_mn + ((kk * 2048) >> 4), idesc_acc, (kk > 0) || (idx > 0));
+          umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, ddo_mn + ((kk * 2048) >> 4), idesc_acc,
+                  (kk > 0) || (idx > 0));
         }
         if (idx + 1 < ni) {  // next block's S^T, into the columns P^T just left
           ok = mbar_wait(&sm.qd_full[st ^ 1], ((idx + 1) >> 1) & 1, wc);
@@ -316,7 +328,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q
-          umma_ts(tDK, tDP + kk * 8, dq_mn + ((kk * 2048) >> 4), idesc_acc, (kk > 0) || (idx > 0));
+          umma_ts(tDK, tDP + (kk >> 2) * 64 + (kk & 3) * 8, dq_mn + ((kk * 2048) >> 4), idesc_acc,
+                  (kk > 0) || (idx > 0));
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // dQ (K = 128 keys) into the dP columns
@@ -334,18 +347,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     __syncwarp();
   }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ key rows: P^T, dS^T
-    regs_set<kLaunchRegs, kBwdRegsKey>();
-    const int r = threadIdx.x;  // key row within the block == TMEM lane
+    regs_set<kBwdLaunchRegs, kBwdRegsKey>();
+    const int g = warp >> 2;          // query half: columns 64g .. 64g+63 of the block
+    const int r = threadIdx.x & 127;  // key row within the block == TMEM lane
     const int kg = j * 128 + r;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tbase + Cfg::kColS + lane_off;
-    const uint32_t tDP = tbase + Cfg::kColDP + lane_off;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tbase + Cfg::kColS + g * 64 + lane_off;
+    const uint32_t tDP = tbase + Cfg::kColDP + g * 64 + lane_off;
     const float sl = scale * kLog2e;
-    const WaitCtx wc{&sm.abort_flag, status, 13};
-    uint8_t* ds_row = sm.ds + (r >> 3) * 1024 + (r & 7) * 128;
     const float2 sl2 = make_float2(sl, sl);
+    const WaitCtx wc{&sm.abort_flag, status, 13};
+    uint8_t* ds_row = sm.ds + g * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
     bool ok = true;
     for (int idx = 0; idx < ni && ok; ++idx) {
       const int st = idx & 1;
@@ -356,17 +370,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       // valid (query q, key k): k < N, and k <= q when causal; q >= N has LSE = +inf -> P = 0
       const bool key_ok = kg < N;
-      const int qlim = (CAUSAL && i == j) ? r : 0;  // on the diagonal block: query index >= r
+      const int qlim = (CAUSAL && i == j) ? r - 64 * g : 0;  // diagonal block: query >= key
       const bool masked = __any_sync(0xffffffffu, !key_ok || qlim > 0);
-      const float* lse2 = sm.lse2[st];
-      const float* dd = sm.dd[st];
-      float pf[128];  // fp32 P^T of this key row, kept for dS
+      const float* lse2 = sm.lse2[st] + 64 * g;
+      const float* dd = sm.dd[st] + 64 * g;
+      // bf16 P^T of this key row for the warpgroup's 64 queries, packed in pairs; dS uses the
+      // same rounded values that enter dV = P^T dO
+      uint32_t pk_all[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
         tmem_ld32(tS + c * 32, sv);
         tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t* pk = pk_all + 16 * c;
 #pragma unroll
         for (int x = 0; x < 32; x += 4) {
           const int ql = c * 32 + x;
@@ -382,14 +398,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!key_ok || ql + 2 < qlim) p2 = 0.f;
             if (!key_ok || ql + 3 < qlim) p3 = 0.f;
           }
-          pf[ql] = p0;
-          pf[ql + 1] = p1;
-          pf[ql + 2] = p2;
-          pf[ql + 3] = p3;
           pk[x / 2] = pack_bf16x2(p0, p1);
           pk[x / 2 + 1] = pack_bf16x2(p2, p3);
         }
-        tmem_st16(tS + c * 16, pk);
+        tmem_st16(tS + c * 16, pk);  // columns already read
       }
       tmem_wait_st();
       tc_fence_before();
@@ -398,7 +410,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t dpv[32];
         tmem_ld32(tDP + c * 32, dpv);
         tmem_wait_ld();
@@ -407,23 +419,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int x = 0; x < 32; x += 4) {
           const int ql = c * 32 + x;
           const float4 d4 = *reinterpret_cast<const float4*>(dd + ql);
-          const float2 a = fmul2(make_float2(pf[ql], pf[ql + 1]),
+          const uint32_t pa = pk_all[ql / 2], pb = pk_all[ql / 2 + 1];
+          const float2 a = fmul2(make_float2(__uint_as_float(pa << 16), __uint_as_float(pa & 0xffff0000u)),
                                  fadd2(make_float2(__uint_as_float(dpv[x]), __uint_as_float(dpv[x + 1])),
                                        make_float2(-d4.x, -d4.y)));
-          const float2 b = fmul2(make_float2(pf[ql + 2], pf[ql + 3]),
+          const float2 b = fmul2(make_float2(__uint_as_float(pb << 16), __uint_as_float(pb & 0xffff0000u)),
                                  fadd2(make_float2(__uint_as_float(dpv[x + 2]), __uint_as_float(dpv[x + 3])),
                                        make_float2(-d4.z, -d4.w)));
           dsk[x / 2] = pack_bf16x2(a.x, a.y);
           dsk[x / 2 + 1] = pack_bf16x2(b.x, b.y);
         }
         tmem_st16(tDP + c * 16, dsk);
-        // dS into shared memory: row r of the 128-byte-swizzled MN-major layout, queries
-        // 32c..32c+31 = four 16-byte units of 64-query chunk c/2
-        uint8_t* base = ds_row + (c >> 1) * 16384;
+        // dS into shared memory: row r of the 128-byte-swizzled MN-major layout; the
+        // warpgroup's 64 queries are chunk g, queries 32c..32c+31 its 16-byte units 4c..4c+3
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
-          const int u = ((c & 1) * 4 + y) ^ (r & 7);
-          *reinterpret_cast<uint4*>(base + u * 16) =
+          const int u = (c * 4 + y) ^ (r & 7);
+          *reinterpret_cast<uint4*>(ds_row + u * 16) =
               make_uint4(dsk[4 * y], dsk[4 * y + 1], dsk[4 * y + 2], dsk[4 * y + 3]);
         }
       }
@@ -432,42 +444,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       mbar_arrive(&sm.ds_ready);
     }
-    // final dK_j, dV_j rows
+    // final rows: warpgroup 0 writes dV_j, warpgroup 1 writes dK_j (x scale)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_done, 0, wc));
     if (ok) {
       tc_fence_after();
-      const uint32_t tDV = tbase + Cfg::kColDV + lane_off;
-      const uint32_t tDK = tbase + Cfg::kColDK + lane_off;
-      const int64_t orow = ((static_cast<int64_t>(b) * N + kg) * H + h) * D;
+      const uint32_t tAcc = tbase + (g == 0 ? Cfg::kColDV : Cfg::kColDK) + lane_off;
+      const float mul = g == 0 ? 1.0f : scale;
+      __nv_bfloat16* dst = (g == 0 ? dv : dk) + ((static_cast<int64_t>(b) * N + kg) * H + h) * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
-        uint32_t a[32], g[32];
-        tmem_ld32(tDV + c, a);
-        tmem_ld32(tDK + c, g);
+        uint32_t a[32];
+        tmem_ld32(tAcc + c, a);
         tmem_wait_ld();
         if (kg < N) {
-          uint4* pv = reinterpret_cast<uint4*>(dv + orow + c);
-          uint4* pk = reinterpret_cast<uint4*>(dk + orow + c);
+          uint4* pv = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            pv[x] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * x]), __uint_as_float(a[8 * x + 1])),
-                               pack_bf16x2(__uint_as_float(a[8 * x + 2]), __uint_as_float(a[8 * x + 3])),
-                               pack_bf16x2(__uint_as_float(a[8 * x + 4]), __uint_as_float(a[8 * x + 5])),
-                               pack_bf16x2(__uint_as_float(a[8 * x + 6]), __uint_as_float(a[8 * x + 7])));
-            pk[x] = make_uint4(
-                pack_bf16x2(__uint_as_float(g[8 * x]) * scale, __uint_as_float(g[8 * x + 1]) * scale),
-                pack_bf16x2(__uint_as_float(g[8 * x + 2]) * scale, __uint_as_float(g[8 * x + 3]) * scale),
-                pack_bf16x2(__uint_as_float(g[8 * x + 4]) * scale, __uint_as_float(g[8 * x + 5]) * scale),
-                pack_bf16x2(__uint_as_float(g[8 * x + 6]) * scale, __uint_as_float(g[8 * x + 7]) * scale));
-          }
+          for (int x = 0; x < 4; ++x)
+            pv[x] = make_uint4(
+                pack_bf16x2(__uint_as_float(a[8 * x]) * mul, __uint_as_float(a[8 * x + 1]) * mul),
+                pack_bf16x2(__uint_as_float(a[8 * x + 2]) * mul, __uint_as_float(a[8 * x + 3]) * mul),
+                pack_bf16x2(__uint_as_float(a[8 * x + 4]) * mul, __uint_as_float(a[8 * x + 5]) * mul),
+                pack_bf16x2(__uint_as_float(a[8 * x + 6]) * mul, __uint_as_float(a[8 * x + 7]) * mul));
         }
       }
     }
     tc_fence_before();
   } else {
-    // ------------------------------------------------------------ dQ drain (warps 4-7)
-    regs_set<kLaunchRegs, kBwdRegsDrain>();
-    const int r = threadIdx.x - 128;  // TMEM lane: head-dim column (d = 128) or query row (d = 64)
+    // ------------------------------------------------------------ dQ drain (warps 8-11)
+    regs_set<kBwdLaunchRegs, kBwdRegsDrain>();
+    const int r = threadIdx.x - 256;  // TMEM lane: head-dim column (d = 128) or query row (d = 64)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tQ = tbase + Cfg::kColDP + lane_off;
     const WaitCtx wc{&sm.abort_flag, status, 14};
@@ -513,7 +518,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }

@@ -76,8 +76,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 /*
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ accumulator
- * [B, H, N, d] followed by the fp32 row sums D_i = sum_x dO_ix O_ix [B, H, N], i.e.
- * 4*B*H*N*(d+1).  Returns 0 for invalid sizes (B, H, N < 1 or d not 64 / 128).
+ * [B, H, N, d], then the fp32 row sums D_i = sum_x dO_ix O_ix and the fp32 LSE_i * log2(e),
+ * each [B*H, Npad] with Npad = N rounded up to a multiple of 128; in total
+ * 4*B*H*(N*d + 2*Npad) bytes.  Returns 0 for invalid sizes (B, H, N < 1 or d not 64 / 128).
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -107,8 +108,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * It performs the same computation as fa_bwd, with the same arguments minus the
  * workspace, and calls no cudaMalloc, cudaFree or other allocating routine.
  *
- * Scratch: a fixed 64 MiB array inside the library (fp32 dQ accumulator and row sums,
- * 4*B*H*N*(d+1) bytes).  Problems that need more return FA_ERR_WORKSPACE and launch
+ * Scratch: a fixed 64 MiB array inside the library holding what fa_bwd's workspace would
+ * (fa_bwd_workspace_size bytes).  Problems that need more return FA_ERR_WORKSPACE and launch
  * nothing; use fa_bwd with a caller-provided workspace for those.  Every GPU that loads
  * the library holds this array until the process exits, whether or not this entry point
  * is used.  All calls on a device share the one array: calls whose work can overlap on

@@ -90,7 +90,7 @@ def test_bwd_validation_codes(lib):
     lib.fa_bwd_workspace_size.argtypes = [ctypes.c_int] * 4
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     ws = lib.fa_bwd_workspace_size(1, 1, 16, 64)
-    assert ws == 16 * 65 * 4
+    assert ws == 4 * (16 * 64 + 2 * 128)
     assert lib.fa_bwd_workspace_size(1, 1, 16, 96) == 0
 
     def call(p=0x10000, wsp=0x10000, wsb=ws, d=64, B=1, scale=0.125):

@@ -72,4 +72,4 @@ def test_bwd_workspace_checks():
     with pytest.raises(api.FAError) as e:
         api.bwd(q, q, q, o, q, lse, workspace=small)
     assert e.value.status == 7
-    assert api.bwd_workspace_size(2, 3, 100, 128) == 2 * 3 * 100 * (128 + 1) * 4
+    assert api.bwd_workspace_size(2, 3, 100, 128) == 4 * 2 * 3 * (100 * 128 + 2 * 128)

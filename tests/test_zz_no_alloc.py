@@ -61,6 +61,6 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     t = {n: x for n in ("q", "k", "v", "o", "do")}
     t["lse"] = torch.zeros(16, dtype=torch.float32, device="cuda")
     B, H, N, d = 1, 64, 2048, 128
-    assert 4 * B * H * N * (d + 1) > NOALLOC_MAX_BYTES
+    assert 4 * B * H * (N * d + 2 * N) > NOALLOC_MAX_BYTES
     rc = _call(fn, t, x, x, x, B, H, N, d, d ** -0.5, True)
     assert rc == 7
