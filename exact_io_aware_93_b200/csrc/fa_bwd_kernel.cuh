@@ -11,7 +11,7 @@
 // Three kernels, one stream:
 //   fa_bwd_pre  : D_i and LSE_i * log2 e (fp32, padded per head to whole 128-row blocks) and
 //                 zeroing of the fp32 dQ accumulator (memory bound)
-//   fa_bwd_main : one CTA per (batch, head, 128-key block j); K_j and V_j stay in shared
+//   fa_bwd_main : one CTA per (batch, head, 128-key block j), head-major; K_j and V_j stay in shared
 //                 memory while 128-query blocks i (i >= j when causal) stream through:
 //                   S^T  = K_j Q_i^T        (tcgen05, both operands in shared memory)
 //                   dP^T = V_j dO_i^T
@@ -190,9 +190,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
   const int nkb = (N + 127) / 128;
   const int BH = B * H;
-  // heavy key blocks first: with causal masking block j meets nkb - j query blocks
-  const int j = blockIdx.x / BH;
-  const int bh = blockIdx.x % BH;
+  // Head-major order: the CTAs resident at any time cover only a few heads, so their dQ
+  // accumulator rows and Q/dO tiles stay in L2.  Within a head, key blocks go heaviest
+  // first (with causal masking block j meets nkb - j query blocks), so the grid ends on
+  // the lightest blocks.
+  const int bh = blockIdx.x / nkb;
+  const int j = blockIdx.x % nkb;
   const int b = bh / H, h = bh % H;
   const int i0 = CAUSAL ? j : 0;
   const int ni = nkb - i0;
