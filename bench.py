@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 
 from exact_io_aware_93_b200.accounting import bwd_flops, fwd_bytes, fwd_flops  # noqa: E402
 from exact_io_aware_93_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+from exact_io_aware_93_b200.replicas import max_over_ranks, whole_job_tflops, world as _world  # noqa: E402
 
 METRIC = "attention fwd/bwd TFLOPS and % of B200 dense-bf16 peak, causal N=2K–128K"
 DEFAULT_WORKLOAD = "causal_fwdbwd_b2_h16_n8192_d128"
@@ -54,11 +55,34 @@ def _peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+def kernel_source_digest() -> str:
+    """Digest of the CUDA sources; ncu traffic figures are valid only for the digest they name."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_93_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, or None if absent or stale."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+    except (OSError, ValueError):
+        return None
+    rec = table.get(kernel, {}).get(workload)
+    if not rec or rec.get("source_digest") != kernel_source_digest():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def _dist_env():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return world, rank, local
+    return _world()
 
 
 class ClockSampler:
@@ -315,26 +339,25 @@ def run_ours(args, w):
     e2e_ms = f0.elapsed_time(f1) / e2e_steps
 
     if world > 1:
-        tt = torch.tensor([ms, e2e_ms, fwd_ms, bwd_ms or 0.0], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, e2e_ms, fwd_ms, bwd_ms = (float(x) for x in tt.tolist())
+        ms, e2e_ms, fwd_ms, bwd_ms = max_over_ranks([ms, e2e_ms, fwd_ms, bwd_ms or 0.0], dev)
         bwd_ms = bwd_ms if with_bwd else None
 
     ff = fwd_flops(w.B, w.H, w.N, w.d, w.causal)
     fb = bwd_flops(w.B, w.H, w.N, w.d, w.causal) if with_bwd else 0.0
     step_flops = ff + fb
-    value = world * step_flops / (ms * 1e-3) / 1e12
-    e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, step_flops, ms)
+    e2e_value = whole_job_tflops(world, step_flops, e2e_ms)
     peak, peak_sus, hbm, peak_kind = _peaks()
     fwd_tf = ff / (fwd_ms * 1e-3) / 1e12
     bwd_tf = fb / (bwd_ms * 1e-3) / 1e12 if with_bwd else None
     # dominant kernel: the one with the larger share of the step
     if with_bwd and bwd_ms > fwd_ms:
-        dom = {"kernel": "fa_bwd (pre + main + post)", "achieved": bwd_tf, "ms": bwd_ms}
+        dom = {"kernel": "fa_bwd (pre + main + post)", "achieved": bwd_tf, "ms": bwd_ms, "key": "fa_bwd"}
     else:
-        dom = {"kernel": "fa_fwd_kernel", "achieved": fwd_tf, "ms": fwd_ms}
+        dom = {"kernel": "fa_fwd_kernel", "achieved": fwd_tf, "ms": fwd_ms, "key": "fa_fwd_kernel"}
     roofline = {"bound": "tensor", "achieved": dom["achieved"], "peak": peak, "unit": "TFLOP/s",
-                "frac": dom["achieved"] / peak, "traffic": None, "kernel": dom["kernel"],
+                "frac": dom["achieved"] / peak, "traffic": measured_traffic(dom["key"], w.name),
+                "kernel": dom["kernel"],
                 "peak_kind": f"{peak_kind} bf16 burst (cuBLAS 8192^3)",
                 "frac_of_sustained": dom["achieved"] / peak_sus,
                 "fwd_alg_bytes": fwd_bytes(w.B, w.H, w.N, w.d)}

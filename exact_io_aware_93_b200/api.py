@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd.restype = i
     L.fa_get_status.argtypes = [vp]
     L.fa_get_status.restype = i
+    L.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+    L.fa_selftest_wait_timeout.restype = i
     L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     L.fa_bwd_workspace_size.restype = ctypes.c_size_t
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
@@ -152,6 +154,12 @@ def get_status(device: torch.device | None = None) -> int:
     """Synchronise the current stream and read-and-clear the device status word."""
     s = torch.cuda.current_stream(device)
     return int(lib().fa_get_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def selftest_wait_timeout(timeout_us: int = 20000) -> int:
+    """Run the bounded-wait self-test on the current stream; returns the launch status."""
+    s = torch.cuda.current_stream()
+    return int(lib().fa_selftest_wait_timeout(int(timeout_us), ctypes.c_void_p(s.cuda_stream)))
 
 
 def attention(q, k, v, causal: bool = False, scale: float | None = None) -> torch.Tensor:

@@ -154,6 +154,23 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   return FA_OK;
 }
 
+// ---------------------------------------------------------------- wait-timeout self-test
+// One warp waits on an mbarrier that nothing will ever arrive on, with the given bound,
+// through the same bounded-wait path the attention kernels use.  The wait runs out, the
+// status word records FA_ERR_TIMEOUT and the kernel returns normally.
+__global__ void fa_wait_timeout_selftest_kernel(uint64_t timeout_ns, int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    fa::mbar_init(&bar, 1);
+    fa::fence_mbar_init();
+  }
+  __syncwarp();
+  const fa::WaitCtx wc{&abort_flag, status, 99};
+  fa::mbar_wait(&bar, 0, wc, timeout_ns);
+}
+
 // ---------------------------------------------------------------- allocation-free backward
 // Scratch for fa_bwd_noalloc: a fixed device array in this module, so callers that may not
 // allocate device memory still get a backward pass.  It exists on every GPU that loads the
@@ -276,6 +293,16 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   const fa_status ss = noalloc_scratch(&scratch);
   if (ss != FA_OK) return ss;
   return fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, scratch, kNoAllocScratchBytes, B, H, N, d, scale, causal, stream);
+}
+
+fa_status fa_selftest_wait_timeout(unsigned int timeout_us, void* stream) {
+  if (timeout_us == 0 || timeout_us > 1000000u) return FA_ERR_INVALID_ARG;
+  DeviceInfo* di = nullptr;
+  const fa_status st = current_device(&di);
+  if (st != FA_OK) return st;
+  fa_wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_us) * 1000u, di->status);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 fa_status fa_get_status(void* stream) {

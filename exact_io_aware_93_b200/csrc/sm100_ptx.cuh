@@ -80,7 +80,8 @@ struct WaitCtx {
 
 // Bounded wait for the phase with the given parity to complete.
 // Returns false (after flagging) on timeout or when another warp has aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                          uint64_t timeout_ns = FA_WAIT_TIMEOUT_NS) {
   const uint32_t a = smem_u32(bar);
   if (mbar_test(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -90,7 +91,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if (++spins >= 32) {
       spins = 0;
       if (*w.abort_flag) return false;
-      if (globaltimer_ns() - t0 > FA_WAIT_TIMEOUT_NS) {
+      if (globaltimer_ns() - t0 > timeout_ns) {
         *w.abort_flag = 1;
         atomicCAS(w.status, 0, 6 /* FA_ERR_TIMEOUT */);
         atomicCAS(w.status + 1, 0, w.site);

@@ -124,6 +124,17 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          int causal, void* stream);
 
 /*
+ * Failure-detection self-test: launches one warp that waits on a barrier nothing will
+ * arrive on, through the same bounded wait the attention kernels use, with a bound of
+ * timeout_us microseconds (1 .. 1000000).  The wait runs out, the kernel records
+ * FA_ERR_TIMEOUT in the device status word and returns; nothing faults or hangs and the
+ * context stays usable.  A following fa_get_status() returns FA_ERR_TIMEOUT.
+ * Returns FA_ERR_INVALID_ARG for a bound out of range, FA_ERR_DEVICE without an sm_100
+ * device, FA_ERR_LAUNCH if the launch fails, else FA_OK.
+ */
+fa_status fa_selftest_wait_timeout(unsigned int timeout_us, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of the
  * current device: FA_OK, or FA_ERR_TIMEOUT if a kernel gave up a bounded wait
  * since the last call.  Returns FA_ERR_DEVICE if the stream or device reports a

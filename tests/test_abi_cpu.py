@@ -105,3 +105,10 @@ def test_bwd_validation_codes(lib):
     assert call(wsp=0) == 7
     assert call(wsb=ws - 1) == 7
     assert call(wsp=0x10004) == 3
+
+
+def test_selftest_validation_without_gpu(lib):
+    lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.c_void_p]
+    lib.fa_selftest_wait_timeout.restype = ctypes.c_int
+    assert lib.fa_selftest_wait_timeout(0, None) == 1
+    assert lib.fa_selftest_wait_timeout(5_000_000, None) == 1
