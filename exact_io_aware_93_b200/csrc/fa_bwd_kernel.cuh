@@ -18,7 +18,7 @@
 //                   P^T  = 2^(S^T * scale * log2 e - LSE_i * log2 e)   (one thread per key)
 //                   dS^T = P^T o (dP^T - D_i)   (with the bf16 P^T that enters dV)
 //                   dV_j += P^T dO_i        (A operand P^T read from tensor memory)
-//                   dK_j += dS^T Q_i        (A operand dS^T read from tensor memory)
+//                   dK_j += dS^T Q_i        (A operand dS^T read from shared memory)
 //                   dQ_i  = dS K_j          (dS written to shared memory, 128-byte swizzle);
 //                                           for d = 128 computed transposed, dQ_i^T = K_j^T dS^T,
 //                                           so that tensor-memory lanes are head-dim columns
@@ -27,13 +27,13 @@
 //                 128-byte lines; dK_j, dV_j are written once at the end.
 //   Per query block the MMA warp issues dP, then (once P is ready) dV and the next block's
 //   S, then (once dS is ready) dK and dQ, so the tensor core works while the key-row
-//   warpgroup computes dS and while the drain empties the previous dQ tile.
+//   warpgroups compute dS and while the drain empties the previous dQ tile.
 //   fa_bwd_post : dQ = bf16(scale * accumulator)
 //
 // Tensor memory (512 columns):
 //   [0,128)   S^T  (fp32).  Key-row warpgroup g (queries 64g..64g+63) reads columns
 //             [64g, 64g+64) and writes its bf16 P^T into [64g, 64g+32), inside its own range.
-//   [128,256) dP^T (fp32), dS^T likewise at [128+64g, 128+64g+32); then dQ_i (or dQ_i^T), fp32
+//   [128,256) dP^T (fp32); once the key rows have read it, dQ_i (or dQ_i^T), fp32
 //   [256,256+D) dV_j accumulator,  [384,384+D) dK_j accumulator
 //
 // Warp roles (512 threads): warps 0-3 and 4-7 key rows for queries 0-63 and 64-127 of the
@@ -171,6 +171,36 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+// P^T for 32 queries of one key row: p = 2^(s * sl - lse2), zero where masked
+// (MASKED: key beyond the sequence, or query index below qlim on the diagonal block);
+// returns the 16 bf16 pairs.  One branch per chunk instead of one per element keeps the
+// unrolled loop a single basic block the compiler can interleave.
+template <bool MASKED>
+__device__ __forceinline__ void bwd_p_chunk(const uint32_t (&sv)[32], const float* lse2, float2 sl2, int q0,
+                                            bool key_ok, int qlim, uint32_t* pk) {
+  float4 l4[8];
+#pragma unroll
+  for (int y = 0; y < 8; ++y) l4[y] = reinterpret_cast<const float4*>(lse2)[y];
+#pragma unroll
+  for (int x = 0; x < 32; x += 4) {
+    const float4 l = l4[x / 4];
+    const float2 a =
+        ffma2(make_float2(__uint_as_float(sv[x]), __uint_as_float(sv[x + 1])), sl2, make_float2(-l.x, -l.y));
+    const float2 b = ffma2(make_float2(__uint_as_float(sv[x + 2]), __uint_as_float(sv[x + 3])), sl2,
+                           make_float2(-l.z, -l.w));
+    float p0 = ex2_approx(a.x), p1 = ex2_approx(a.y), p2 = ex2_approx(b.x), p3 = ex2_approx(b.y);
+    if (MASKED) {
+      const int ql = q0 + x;
+      p0 = (key_ok && ql >= qlim) ? p0 : 0.f;
+      p1 = (key_ok && ql + 1 >= qlim) ? p1 : 0.f;
+      p2 = (key_ok && ql + 2 >= qlim) ? p2 : 0.f;
+      p3 = (key_ok && ql + 3 >= qlim) ? p3 : 0.f;
+    }
+    pk[x / 2] = pack_bf16x2(p0, p1);
+    pk[x / 2 + 1] = pack_bf16x2(p2, p3);
+  }
+}
+
 // ---------------------------------------------------------------- main
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -276,12 +306,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       const WaitCtx wc{&sm.abort_flag, status, 12};
       constexpr uint32_t idesc_sdp = idesc_bf16(128, 128, 0, 0);  // K-major x K-major
-      constexpr uint32_t idesc_acc = idesc_bf16(128, D, 0, 1);    // TMEM A x MN-major B
+      constexpr uint32_t idesc_acc = idesc_bf16(128, D, 0, 1);    // K-major (TMEM or smem) A x MN-major B
       constexpr uint32_t idesc_dq = idesc_bf16(128, D, 1, 1);     // MN-major A (dS) x MN-major B (K)
       const uint64_t dk_kmaj = sdesc_sw128(smem_u32(sm.k), 16, 1024);
       const uint64_t dv_kmaj = sdesc_sw128(smem_u32(sm.v), 16, 1024);
       const uint64_t dk_mn = sdesc_sw128(smem_u32(sm.k), Cfg::kChunkBytes, 1024);
-      const uint64_t dds = sdesc_sw128(smem_u32(sm.ds), 128 * 128, 1024);
+      const uint64_t dds = sdesc_sw128(smem_u32(sm.ds), 128 * 128, 1024);  // dS^T as MN-major operand
+      // the same buffer read as K-major rows (key k, queries contiguous): the A operand dS^T of dK
+      const uint64_t dds_k = sdesc_sw128(smem_u32(sm.ds), 16, 1024);
       const uint32_t tS = tbase + Cfg::kColS, tDP = tbase + Cfg::kColDP;
       const uint32_t tDV = tbase + Cfg::kColDV, tDK = tbase + Cfg::kColDK;
       auto kmaj_gemm = [&](uint32_t tD, uint64_t da, uint64_t db) {  // (128 x d) . (128 x d)^T
@@ -330,9 +362,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q
-          umma_ts(tDK, tDP + (kk >> 2) * 64 + (kk & 3) * 8, dq_mn + ((kk * 2048) >> 4), idesc_acc,
-                  (kk > 0) || (idx > 0));
+        for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q, dS^T read K-major from shared memory
+          const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4;
+          umma_ss(tDK, dds_k + off, dq_mn + ((kk * 2048) >> 4), idesc_acc, (kk > 0) || (idx > 0));
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // dQ (K = 128 keys) into the dP columns
@@ -386,24 +418,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(tS + c * 32, sv);
         tmem_wait_ld();
         uint32_t* pk = pk_all + 16 * c;
-#pragma unroll
-        for (int x = 0; x < 32; x += 4) {
-          const int ql = c * 32 + x;
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + ql);
-          const float2 a = ffma2(make_float2(__uint_as_float(sv[x]), __uint_as_float(sv[x + 1])), sl2,
-                                 make_float2(-l4.x, -l4.y));
-          const float2 b = ffma2(make_float2(__uint_as_float(sv[x + 2]), __uint_as_float(sv[x + 3])), sl2,
-                                 make_float2(-l4.z, -l4.w));
-          float p0 = ex2_approx(a.x), p1 = ex2_approx(a.y), p2 = ex2_approx(b.x), p3 = ex2_approx(b.y);
-          if (masked) {
-            if (!key_ok || ql < qlim) p0 = 0.f;
-            if (!key_ok || ql + 1 < qlim) p1 = 0.f;
-            if (!key_ok || ql + 2 < qlim) p2 = 0.f;
-            if (!key_ok || ql + 3 < qlim) p3 = 0.f;
-          }
-          pk[x / 2] = pack_bf16x2(p0, p1);
-          pk[x / 2 + 1] = pack_bf16x2(p2, p3);
-        }
+        if (masked)
+          bwd_p_chunk<true>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, pk);
+        else
+          bwd_p_chunk<false>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, pk);
         tmem_st16(tS + c * 16, pk);  // columns already read
       }
       tmem_wait_st();
@@ -418,10 +436,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(tDP + c * 32, dpv);
         tmem_wait_ld();
         uint32_t dsk[16];
+        float4 d4s[8];
+#pragma unroll
+        for (int y = 0; y < 8; ++y) d4s[y] = reinterpret_cast<const float4*>(dd + c * 32)[y];
 #pragma unroll
         for (int x = 0; x < 32; x += 4) {
           const int ql = c * 32 + x;
-          const float4 d4 = *reinterpret_cast<const float4*>(dd + ql);
+          const float4 d4 = d4s[x / 4];
           const uint32_t pa = pk_all[ql / 2], pb = pk_all[ql / 2 + 1];
           const float2 a = fmul2(make_float2(__uint_as_float(pa << 16), __uint_as_float(pa & 0xffff0000u)),
                                  fadd2(make_float2(__uint_as_float(dpv[x]), __uint_as_float(dpv[x + 1])),
@@ -432,7 +453,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           dsk[x / 2] = pack_bf16x2(a.x, a.y);
           dsk[x / 2 + 1] = pack_bf16x2(b.x, b.y);
         }
-        tmem_st16(tDP + c * 16, dsk);
         // dS into shared memory: row r of the 128-byte-swizzled MN-major layout; the
         // warpgroup's 64 queries are chunk g, queries 32c..32c+31 its 16-byte units 4c..4c+3
 #pragma unroll
@@ -442,7 +462,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               make_uint4(dsk[4 * y], dsk[4 * y + 1], dsk[4 * y + 2], dsk[4 * y + 3]);
         }
       }
-      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sm.ds_ready);
