@@ -26,6 +26,10 @@
  * "Flash Attention vs Standard Attention", section "Engineering
  * Perspective"): key j is visible to query i iff j <= i.  Sequence lengths of
  * queries and keys are equal, so top-left and bottom-right alignment agree.
+ * A sliding window ("Flash Attention Explained", institutepm.com, "Sliding Window
+ * Attention": each token only attends to nearby tokens) further limits causal
+ * attention to the last `window` + 1 keys: j visible to i iff i - window <= j <= i.
+ * window < 0 means no window.
  *
  * LSE_i = ln sum_j exp(S_ij) over visible j (natural log), the per-row
  * statistic the backward pass recomputes from.
@@ -63,8 +67,10 @@
 #include <omp.h>
 #endif
 
-static int n_visible(int64_t i, int64_t N, int causal) {
-    return (int)(causal ? (i + 1) : N);
+/* Visible keys of query i: [lo, hi). */
+static void visible_range(int64_t i, int64_t N, int causal, int64_t window, int64_t* lo, int64_t* hi) {
+    *hi = causal ? (i + 1) : N;
+    *lo = (window >= 0 && i - window > 0) ? (i - window) : 0;
 }
 
 static double dot(const double* a, const double* b, int d) {
@@ -73,13 +79,16 @@ static double dot(const double* a, const double* b, int d) {
     return s;
 }
 
-/* Scores of row i against every visible key, into srow[0..nv). Returns nv. */
-static int score_row(const double* q, const double* k, int64_t N, int d,
-                     double scale, int causal, int64_t i, double* srow) {
-    int nv = n_visible(i, N, causal);
+/* Scores of row i against every visible key, into srow[0..nv) for keys lo..lo+nv-1.
+ * Returns nv and stores lo. */
+static int score_row(const double* q, const double* k, int64_t N, int d, double scale, int causal,
+                     int64_t window, int64_t i, double* srow, int64_t* lo_out) {
+    int64_t lo, hi;
+    visible_range(i, N, causal, window, &lo, &hi);
     const double* qi = q + i * d;
-    for (int j = 0; j < nv; ++j) srow[j] = scale * dot(qi, k + (int64_t)j * d, d);
-    return nv;
+    for (int64_t j = lo; j < hi; ++j) srow[j - lo] = scale * dot(qi, k + j * d, d);
+    *lo_out = lo;
+    return (int)(hi - lo);
 }
 
 /* Two-pass log-sum-exp of srow[0..nv): max first, then sum of exp(s - max). */
@@ -112,10 +121,11 @@ void oracle_set_num_threads(int n) {
  * rows[r] in [0, N); o_out is [n_rows][d]; lse_out is [n_rows].
  */
 int oracle_fwd_rows(const double* q, const double* k, const double* v,
-                    int64_t N, int d, double scale, int causal,
+                    int64_t N, int d, double scale, int causal, int64_t window,
                     const int64_t* rows, int64_t n_rows,
                     double* o_out, double* lse_out) {
     if (!q || !k || !v || !rows || !o_out || !lse_out || N < 1 || d < 1) return -1;
+    if (window >= 0 && !causal) return -1;
     for (int64_t r = 0; r < n_rows; ++r)
         if (rows[r] < 0 || rows[r] >= N) return -1;
     int err = 0;
@@ -128,14 +138,14 @@ int oracle_fwd_rows(const double* q, const double* k, const double* v,
         } else {
 #pragma omp for schedule(dynamic, 4)
             for (int64_t r = 0; r < n_rows; ++r) {
-                int64_t i = rows[r];
-                int nv = score_row(q, k, N, d, scale, causal, i, srow);
+                int64_t i = rows[r], lo;
+                int nv = score_row(q, k, N, d, scale, causal, window, i, srow, &lo);
                 double lse = lse_two_pass(srow, nv);
                 double* o = o_out + r * d;
                 for (int x = 0; x < d; ++x) o[x] = 0.0;
                 for (int j = 0; j < nv; ++j) {
                     double p = exp(srow[j] - lse);
-                    const double* vj = v + (int64_t)j * d;
+                    const double* vj = v + (lo + j) * d;
                     for (int x = 0; x < d; ++x) o[x] += p * vj[x];
                 }
                 lse_out[r] = lse;
@@ -152,13 +162,15 @@ int oracle_fwd_rows(const double* q, const double* k, const double* v,
  * the softmax itself (rows sum to one, agreement with a library softmax).
  */
 int oracle_prob_row(const double* q, const double* k, int64_t N, int d,
-                    double scale, int causal, int64_t i, double* p_out) {
+                    double scale, int causal, int64_t window, int64_t i, double* p_out) {
     if (!q || !k || !p_out || N < 1 || d < 1 || i < 0 || i >= N) return -1;
+    if (window >= 0 && !causal) return -1;
     double* srow = (double*)malloc(sizeof(double) * (size_t)N);
     if (!srow) return -2;
-    int nv = score_row(q, k, N, d, scale, causal, i, srow);
+    int64_t lo;
+    int nv = score_row(q, k, N, d, scale, causal, window, i, srow, &lo);
     double lse = lse_two_pass(srow, nv);
-    for (int64_t j = 0; j < N; ++j) p_out[j] = (j < nv) ? exp(srow[j] - lse) : 0.0;
+    for (int64_t j = 0; j < N; ++j) p_out[j] = (j >= lo && j < lo + nv) ? exp(srow[j - lo] - lse) : 0.0;
     free(srow);
     return 0;
 }
@@ -173,10 +185,11 @@ int oracle_prob_row(const double* q, const double* k, int64_t N, int d,
  * blocked or reordered beyond the definitions in the file header.
  */
 int oracle_bwd_rows(const double* q, const double* k, const double* v,
-                    const double* dO, int64_t N, int d, double scale, int causal,
+                    const double* dO, int64_t N, int d, double scale, int causal, int64_t window,
                     const int64_t* qrows, int64_t nq, double* dq_out, double* c_out,
                     const int64_t* krows, int64_t nk, double* dk_out, double* dv_out) {
     if (!q || !k || !v || !dO || N < 1 || d < 1) return -1;
+    if (window >= 0 && !causal) return -1;
     if (nq > 0 && (!qrows || !dq_out)) return -1;
     if (nk > 0 && (!krows || !dk_out || !dv_out)) return -1;
     for (int64_t r = 0; r < nq; ++r) if (qrows[r] < 0 || qrows[r] >= N) return -1;
@@ -197,13 +210,14 @@ int oracle_bwd_rows(const double* q, const double* k, const double* v,
         } else {
 #pragma omp for schedule(dynamic, 8)
             for (int64_t i = 0; i < N; ++i) {
-                int nv = score_row(q, k, N, d, scale, causal, i, srow);
+                int64_t lo;
+                int nv = score_row(q, k, N, d, scale, causal, window, i, srow, &lo);
                 double l = lse_two_pass(srow, nv);
                 double c = 0.0;
                 const double* doi = dO + i * d;
                 for (int j = 0; j < nv; ++j) {
                     double p = exp(srow[j] - l);
-                    double dp = dot(doi, v + (int64_t)j * d, d);
+                    double dp = dot(doi, v + (lo + j) * d, d);
                     c += p * dp;
                 }
                 lse[i] = l;
@@ -217,16 +231,16 @@ int oracle_bwd_rows(const double* q, const double* k, const double* v,
     /* dQ_i = scale * sum_j dS_ij k_j at the requested query rows. */
 #pragma omp parallel for schedule(dynamic, 4)
     for (int64_t r = 0; r < nq; ++r) {
-        int64_t i = qrows[r];
-        int nv = n_visible(i, N, causal);
+        int64_t i = qrows[r], lo, hi;
+        visible_range(i, N, causal, window, &lo, &hi);
         const double* qi = q + i * d;
         const double* doi = dO + i * d;
         double* dq = dq_out + r * d;
         for (int x = 0; x < d; ++x) dq[x] = 0.0;
-        for (int j = 0; j < nv; ++j) {
-            const double* kj = k + (int64_t)j * d;
+        for (int64_t j = lo; j < hi; ++j) {
+            const double* kj = k + j * d;
             double p = exp(scale * dot(qi, kj, d) - lse[i]);
-            double ds = p * (dot(doi, v + (int64_t)j * d, d) - crow[i]);
+            double ds = p * (dot(doi, v + j * d, d) - crow[i]);
             for (int x = 0; x < d; ++x) dq[x] += ds * kj[x];
         }
         for (int x = 0; x < d; ++x) dq[x] *= scale;
@@ -242,8 +256,10 @@ int oracle_bwd_rows(const double* q, const double* k, const double* v,
         double* dk = dk_out + r * d;
         double* dv = dv_out + r * d;
         for (int x = 0; x < d; ++x) { dk[x] = 0.0; dv[x] = 0.0; }
+        /* queries that see key j: i >= j when causal, and i <= j + window with a window */
         int64_t i0 = causal ? j : 0;
-        for (int64_t i = i0; i < N; ++i) {
+        int64_t i1 = (window >= 0 && j + window + 1 < N) ? (j + window + 1) : N;
+        for (int64_t i = i0; i < i1; ++i) {
             const double* qi = q + i * d;
             const double* doi = dO + i * d;
             double p = exp(scale * dot(qi, kj, d) - lse[i]);

@@ -73,13 +73,13 @@ def _load():
     path = build_oracle()
     lib = ctypes.CDLL(path)
     lib.oracle_fwd_rows.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int, ctypes.c_double,
-                                    ctypes.c_int, _ip, ctypes.c_int64, _dp, _dp]
+                                    ctypes.c_int, ctypes.c_int64, _ip, ctypes.c_int64, _dp, _dp]
     lib.oracle_fwd_rows.restype = ctypes.c_int
     lib.oracle_prob_row.argtypes = [_dp, _dp, ctypes.c_int64, ctypes.c_int, ctypes.c_double,
-                                    ctypes.c_int, ctypes.c_int64, _dp]
+                                    ctypes.c_int, ctypes.c_int64, ctypes.c_int64, _dp]
     lib.oracle_prob_row.restype = ctypes.c_int
     lib.oracle_bwd_rows.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int64, ctypes.c_int,
-                                    ctypes.c_double, ctypes.c_int,
+                                    ctypes.c_double, ctypes.c_int, ctypes.c_int64,
                                     _ip, ctypes.c_int64, _dp, _dp,
                                     _ip, ctypes.c_int64, _dp, _dp]
     lib.oracle_bwd_rows.restype = ctypes.c_int
@@ -114,8 +114,10 @@ def _check_head(q, k, v):
         raise ValueError(f"one head of shape [N, d] expected, got {q.shape}, {k.shape}, {v.shape}")
 
 
-def fwd_rows(q, k, v, scale: float, causal: bool, rows=None):
-    """O (fp64 [len(rows), d]) and LSE (fp64 [len(rows)]) of one head at the given query rows."""
+def fwd_rows(q, k, v, scale: float, causal: bool, rows=None, window: int = -1):
+    """O (fp64 [len(rows), d]) and LSE (fp64 [len(rows)]) of one head at the given query rows.
+
+    window >= 0 (causal only): query i sees keys i - window .. i."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     _check_head(q, k, v)
     n, d = q.shape
@@ -123,26 +125,26 @@ def fwd_rows(q, k, v, scale: float, causal: bool, rows=None):
     o = np.empty((rows.size, d), np.float64)
     lse = np.empty(rows.size, np.float64)
     rc = _load().oracle_fwd_rows(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), n, d, float(scale),
-                                 int(bool(causal)), _ptr(rows, _ip), rows.size,
+                                 int(bool(causal)), int(window), _ptr(rows, _ip), rows.size,
                                  _ptr(o, _dp), _ptr(lse, _dp))
     if rc != 0:
         raise RuntimeError(f"oracle_fwd_rows failed ({rc})")
     return o, lse
 
 
-def prob_row(q, k, scale: float, causal: bool, i: int) -> np.ndarray:
+def prob_row(q, k, scale: float, causal: bool, i: int, window: int = -1) -> np.ndarray:
     """The normalised attention probabilities P_i. of one query row (zeros where masked)."""
     q, k = _f64(q), _f64(k)
     n, d = q.shape
     p = np.empty(n, np.float64)
     rc = _load().oracle_prob_row(_ptr(q, _dp), _ptr(k, _dp), n, d, float(scale),
-                                 int(bool(causal)), int(i), _ptr(p, _dp))
+                                 int(bool(causal)), int(window), int(i), _ptr(p, _dp))
     if rc != 0:
         raise RuntimeError(f"oracle_prob_row failed ({rc})")
     return p
 
 
-def bwd_rows(q, k, v, do, scale: float, causal: bool, qrows=None, krows=None):
+def bwd_rows(q, k, v, do, scale: float, causal: bool, qrows=None, krows=None, window: int = -1):
     """Gradients of L = sum(O * dO) for one head.
 
     Returns (dq [len(qrows), d], c [len(qrows)], dk [len(krows), d], dv [len(krows), d]),
@@ -158,7 +160,7 @@ def bwd_rows(q, k, v, do, scale: float, causal: bool, qrows=None, krows=None):
     dk = np.empty((krows.size, d), np.float64)
     dv = np.empty((krows.size, d), np.float64)
     rc = _load().oracle_bwd_rows(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(do, _dp), n, d,
-                                 float(scale), int(bool(causal)),
+                                 float(scale), int(bool(causal)), int(window),
                                  _ptr(qrows, _ip), qrows.size, _ptr(dq, _dp), _ptr(c, _dp),
                                  _ptr(krows, _ip), krows.size, _ptr(dk, _dp), _ptr(dv, _dp))
     if rc != 0:
@@ -166,18 +168,21 @@ def bwd_rows(q, k, v, do, scale: float, causal: bool, qrows=None, krows=None):
     return dq, c, dk, dv
 
 
-def _visible(n: int, causal: bool) -> np.ndarray:
-    if causal:
-        return np.tril(np.ones((n, n), dtype=bool))
-    return np.ones((n, n), dtype=bool)
+def _visible(n: int, causal: bool, window: int = -1) -> np.ndarray:
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    vis = (j <= i) if causal else np.ones((n, n), dtype=bool)
+    if window >= 0:
+        vis = vis & (j >= i - window)
+    return vis
 
 
-def dense_fwd(q, k, v, scale: float, causal: bool):
+def dense_fwd(q, k, v, scale: float, causal: bool, window: int = -1):
     """Whole-matrix fp64 standard attention of one head: (O [N, d], LSE [N], P [N, N])."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     n = q.shape[0]
     s = scale * (q @ k.T)
-    s = np.where(_visible(n, causal), s, -np.inf)
+    s = np.where(_visible(n, causal, window), s, -np.inf)
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m)
     l = e.sum(axis=1, keepdims=True)
@@ -185,17 +190,17 @@ def dense_fwd(q, k, v, scale: float, causal: bool):
     return p @ v, (m + np.log(l))[:, 0], p
 
 
-def dense_bwd(q, k, v, do, scale: float, causal: bool):
+def dense_bwd(q, k, v, do, scale: float, causal: bool, window: int = -1):
     """Whole-matrix fp64 gradients of L = sum(O * dO): (dQ, dK, dV, c)."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
-    _, _, p = dense_fwd(q, k, v, scale, causal)
+    _, _, p = dense_fwd(q, k, v, scale, causal, window)
     dp = do @ v.T
     c = (p * dp).sum(axis=1)
     ds = p * (dp - c[:, None])
     return scale * (ds @ k), scale * (ds.T @ q), p.T @ do, c
 
 
-def online_fwd(q, k, v, scale: float, causal: bool, tile_widths):
+def online_fwd(q, k, v, scale: float, causal: bool, tile_widths, window: int = -1):
     """Streaming (online-softmax) forward of one head, keys consumed in tiles of the given widths.
 
     State per query row: running maximum m, running sum l of exp(s - m), and an
@@ -208,7 +213,7 @@ def online_fwd(q, k, v, scale: float, causal: bool, tile_widths):
     widths = [int(w) for w in tile_widths]
     if sum(widths) != n or min(widths) < 1:
         raise ValueError("tile widths must be positive and cover all keys")
-    vis = _visible(n, causal)
+    vis = _visible(n, causal, window)
     m = np.full(n, -np.inf)
     l = np.zeros(n)
     acc = np.zeros((n, d))

@@ -192,3 +192,86 @@ ALL_FWD_CHECKS = [check_library_softmax, check_n1_closed_form, check_n2_logistic
                   check_rows_sum_to_one, check_identical_scores, check_dominant_score,
                   check_causal_future_blind]
 ALL_BWD_CHECKS = [check_finite_differences, check_gradient_invariants]
+
+
+# ---------------------------------------------------------------- sliding window (causal)
+# An implementation for these checks takes `window` as a keyword: query i sees keys
+# i - window .. i.
+
+def check_window_library_softmax(impl, seed=21):
+    """Brute force with a window mask against scipy's softmax and logsumexp."""
+    rng = _rng(seed)
+    for trial in range(10):
+        n = int(rng.integers(1, 17))
+        d = int(rng.integers(1, 7))
+        window = int(rng.integers(0, 6))
+        scale = float(rng.uniform(0.2, 1.2))
+        q, k, v = (_bf16_grid(rng.standard_normal((n, d))) for _ in range(3))
+        o, lse = impl.fwd(q, k, v, scale, True, window=window)
+        for i in range(n):
+            js = list(range(max(0, i - window), i + 1))
+            s = np.array([scale * sum(q[i, x] * k[j, x] for x in range(d)) for j in js])
+            p = softmax(s)
+            o_ref = sum(pp * v[j] for pp, j in zip(p, js))
+            np.testing.assert_allclose(o[i], o_ref, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse[i], logsumexp(s), rtol=1e-13, atol=1e-13)
+
+
+def check_window_zero_closed_form(impl, seed=22):
+    """window = 0: every query sees only itself, so O_i = v_i and LSE_i = S_ii."""
+    rng = _rng(seed)
+    n, d = 12, 5
+    q, k, v = (_bf16_grid(rng.standard_normal((n, d))) for _ in range(3))
+    o, lse = impl.fwd(q, k, v, 0.7, True, window=0)
+    assert np.array_equal(o, v)
+    np.testing.assert_allclose(lse, 0.7 * (q * k).sum(axis=1), rtol=0, atol=1e-14)
+    dq, dk, dv, _ = impl.bwd(q, k, v, q, 0.7, True, window=0)
+    np.testing.assert_allclose(dq, 0.0, atol=1e-15)
+    np.testing.assert_allclose(dk, 0.0, atol=1e-15)
+    np.testing.assert_allclose(dv, q, rtol=0, atol=1e-15)  # dO = q here: dV_j = dO_j
+
+
+def check_window_past_blind(impl, seed=23):
+    """Keys older than the window do not matter: changing them leaves O_i bit-identical,
+    and a window reaching the first key equals plain causal attention."""
+    rng = _rng(seed)
+    n, d, w = 30, 6, 4
+    q, k, v = (_bf16_grid(rng.standard_normal((n, d))) for _ in range(3))
+    o, lse = impl.fwd(q, k, v, 0.5, True, window=w)
+    i0 = 20
+    k2, v2 = k.copy(), v.copy()
+    k2[: i0 - w] = _bf16_grid(rng.standard_normal((i0 - w, d)) * 4)
+    v2[: i0 - w] = 9.0
+    o2, lse2 = impl.fwd(q, k2, v2, 0.5, True, window=w)
+    assert np.array_equal(o[i0:], o2[i0:]) and np.array_equal(lse[i0:], lse2[i0:])
+    assert not np.array_equal(o[: i0 - 1], o2[: i0 - 1])
+    oc, lc = impl.fwd(q, k, v, 0.5, True)
+    ow, lw = impl.fwd(q, k, v, 0.5, True, window=n - 1)
+    np.testing.assert_allclose(ow, oc, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lw, lc, rtol=0, atol=1e-14)
+
+
+def check_window_finite_differences(impl, seed=24, h=1e-6):
+    """Central finite differences of L = sum(O * dO) with a window."""
+    rng = _rng(seed)
+    n, d, w = 7, 3, 2
+    q, k, v, do = (rng.standard_normal((n, d)) for _ in range(4))
+    dq, dk, dv, _ = impl.bwd(q, k, v, do, 0.8, True, window=w)
+
+    def loss(args):
+        o, _ = impl.fwd(args["q"], args["k"], args["v"], 0.8, True, window=w)
+        return float((o * do).sum())
+
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += h
+            minus[idx] -= h
+            num[idx] = (loss({"q": q, "k": k, "v": v, name: plus})
+                        - loss({"q": q, "k": k, "v": v, name: minus})) / (2 * h)
+        np.testing.assert_allclose(grad, num, rtol=0, atol=2e-7, err_msg=f"d{name} (window)")
+
+
+ALL_WINDOW_CHECKS = [check_window_library_softmax, check_window_zero_closed_form,
+                     check_window_past_blind, check_window_finite_differences]

@@ -10,11 +10,13 @@ from tests import oracle_pins as pins
 
 
 def _fwd(q, k, v, scale, causal, *, use_scale=True, mask_shift=0, lse_no_max=False,
-         reverse_v=False, no_norm=False):
+         reverse_v=False, no_norm=False, window=-1, window_shift=0):
     q, k, v = (np.asarray(a, np.float64) for a in (q, k, v))
     n = q.shape[0]
     s = (scale if use_scale else 1.0) * (q @ k.T)
     vis = np.tril(np.ones((n, n), bool), k=mask_shift) if causal else np.ones((n, n), bool)
+    if window >= 0:
+        vis = vis & ~np.tril(np.ones((n, n), bool), k=-(window + 1 + window_shift))
     s = np.where(vis, s, -np.inf)
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m)
@@ -26,9 +28,9 @@ def _fwd(q, k, v, scale, causal, *, use_scale=True, mask_shift=0, lse_no_max=Fal
 
 
 def _bwd(q, k, v, do, scale, causal, *, sign=1.0, c_from_dp=False, dk_scale=True,
-         dv_untransposed=False, fwd_kw=None):
+         dv_untransposed=False, fwd_kw=None, window=-1):
     q, k, v, do = (np.asarray(a, np.float64) for a in (q, k, v, do))
-    _, _, p = _fwd(q, k, v, scale, causal, **(fwd_kw or {}))
+    _, _, p = _fwd(q, k, v, scale, causal, window=window, **(fwd_kw or {}))
     dp = do @ v.T
     c = dp.sum(axis=1) if c_from_dp else (p * dp).sum(axis=1)
     ds = sign * p * (dp - c[:, None])
@@ -42,13 +44,13 @@ def _impl(fwd_kw=None, bwd_kw=None):
 
     class Mutant:
         @staticmethod
-        def fwd(q, k, v, scale, causal):
-            o, lse, _ = _fwd(q, k, v, scale, causal, **fwd_kw)
+        def fwd(q, k, v, scale, causal, window=-1):
+            o, lse, _ = _fwd(q, k, v, scale, causal, window=window, **fwd_kw)
             return o, lse
 
         @staticmethod
-        def bwd(q, k, v, do, scale, causal):
-            return _bwd(q, k, v, do, scale, causal, fwd_kw=fwd_kw, **bwd_kw)
+        def bwd(q, k, v, do, scale, causal, window=-1):
+            return _bwd(q, k, v, do, scale, causal, fwd_kw=fwd_kw, window=window, **bwd_kw)
     return Mutant
 
 
@@ -63,11 +65,13 @@ MUTANTS = {
     "row_constant_from_dp_only": _impl(bwd_kw={"c_from_dp": True}),
     "dk_missing_scale": _impl(bwd_kw={"dk_scale": False}),
     "dv_untransposed": _impl(bwd_kw={"dv_untransposed": True}),
+    "window_one_key_too_many": _impl(fwd_kw={"window_shift": 1}),
+    "window_one_key_too_few": _impl(fwd_kw={"window_shift": -1}),
 }
 
 
 def _fails_some_pin(impl):
-    for check in pins.ALL_FWD_CHECKS + pins.ALL_BWD_CHECKS:
+    for check in pins.ALL_FWD_CHECKS + pins.ALL_BWD_CHECKS + pins.ALL_WINDOW_CHECKS:
         try:
             with np.errstate(all="ignore"):
                 check(impl)

@@ -15,38 +15,38 @@ class COracle:
     """The C oracle (full rows) seen through the pin interface."""
 
     @staticmethod
-    def fwd(q, k, v, scale, causal):
-        return oracle.fwd_rows(q, k, v, scale, causal)
+    def fwd(q, k, v, scale, causal, window=-1):
+        return oracle.fwd_rows(q, k, v, scale, causal, window=window)
 
     @staticmethod
-    def bwd(q, k, v, do, scale, causal):
-        dq, c, dk, dv = oracle.bwd_rows(q, k, v, do, scale, causal)
+    def bwd(q, k, v, do, scale, causal, window=-1):
+        dq, c, dk, dv = oracle.bwd_rows(q, k, v, do, scale, causal, window=window)
         return dq, dk, dv, c
 
 
 class DenseOracle:
     @staticmethod
-    def fwd(q, k, v, scale, causal):
-        o, lse, _ = oracle.dense_fwd(q, k, v, scale, causal)
+    def fwd(q, k, v, scale, causal, window=-1):
+        o, lse, _ = oracle.dense_fwd(q, k, v, scale, causal, window)
         return o, lse
 
     @staticmethod
-    def bwd(q, k, v, do, scale, causal):
-        return oracle.dense_bwd(q, k, v, do, scale, causal)
+    def bwd(q, k, v, do, scale, causal, window=-1):
+        return oracle.dense_bwd(q, k, v, do, scale, causal, window)
 
 
 class OnlineOracle:
     """The streaming form, keys in uneven tiles; backward borrowed from the dense twin."""
 
     @staticmethod
-    def fwd(q, k, v, scale, causal):
+    def fwd(q, k, v, scale, causal, window=-1):
         n = np.asarray(q).shape[0]
         widths, left, w = [], n, 1
         while left:
             widths.append(min(w, left))
             left -= widths[-1]
             w = w % 5 + 2
-        return oracle.online_fwd(q, k, v, scale, causal, widths)
+        return oracle.online_fwd(q, k, v, scale, causal, widths, window)
 
     bwd = DenseOracle.bwd
 
@@ -64,6 +64,31 @@ def test_forward_pins(impl, check):
 @pytest.mark.parametrize("check", pins.ALL_BWD_CHECKS, ids=lambda f: f.__name__)
 def test_backward_pins(impl, check):
     check(IMPLS[impl])
+
+
+@pytest.mark.parametrize("impl", sorted(IMPLS))
+@pytest.mark.parametrize("check", pins.ALL_WINDOW_CHECKS, ids=lambda f: f.__name__)
+def test_window_pins(impl, check):
+    if impl == "online" and check is pins.check_window_finite_differences:
+        pytest.skip("the streaming form has no backward of its own")
+    check(IMPLS[impl])
+
+
+def test_c_oracle_window_sampled_rows_and_bad_args():
+    rng = np.random.default_rng(31)
+    n, d = 200, 8
+    q, k, v, do = (rng.standard_normal((n, d)) for _ in range(4))
+    rows = np.array([0, 3, 64, 199])
+    o_all, l_all = oracle.fwd_rows(q, k, v, 0.3, True, window=17)
+    o, l = oracle.fwd_rows(q, k, v, 0.3, True, rows, window=17)
+    assert np.array_equal(o, o_all[rows]) and np.array_equal(l, l_all[rows])
+    dq_all, c_all, dk_all, dv_all = oracle.bwd_rows(q, k, v, do, 0.3, True, window=17)
+    dq, c, dk, dv = oracle.bwd_rows(q, k, v, do, 0.3, True, rows, rows, window=17)
+    assert np.array_equal(dk, dk_all[rows]) and np.array_equal(dq, dq_all[rows])
+    p = oracle.prob_row(q, k, 0.3, True, 100, window=17)
+    assert abs(p.sum() - 1) < 1e-14 and np.all(p[:83] == 0) and np.all(p[101:] == 0)
+    with pytest.raises(RuntimeError):
+        oracle.fwd_rows(q, k, v, 0.3, False, window=5)   # a window needs causal attention
 
 
 def test_prob_row_matches_library_softmax():
