@@ -35,8 +35,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from exact_io_aware_93_b200.accounting import bwd_flops, fwd_bytes, fwd_flops  # noqa: E402
-from exact_io_aware_93_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+from exact_io_aware_93_b200.accounting import bwd_flops_window, fwd_bytes, fwd_flops_window  # noqa: E402
+from exact_io_aware_93_b200.inputs import EXTRA_WORKLOADS, WORKLOADS, make_inputs  # noqa: E402
 from exact_io_aware_93_b200.replicas import max_over_ranks, whole_job_tflops, world as _world  # noqa: E402
 
 METRIC = "attention fwd/bwd TFLOPS and % of B200 dense-bf16 peak, causal N=2K–128K"
@@ -153,13 +153,25 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def _win(w):
+    return None if w.window < 0 else w.window
+
+
+def fwd_flops(B, H, N, d, causal, window=-1):
+    return fwd_flops_window(B, H, N, d, causal, window)
+
+
+def bwd_flops(B, H, N, d, causal, window=-1):
+    return bwd_flops_window(B, H, N, d, causal, window)
+
+
 def _step_fn(api, t, w, with_bwd, events=None):
     """One pass of the hot path: fa_fwd then (if available) fa_bwd, on the current stream."""
     def step():
         if events is not None:
             events["fwd"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
             events["fwd"][-1][0].record()
-        api.fwd(t["q"], t["k"], t["v"], causal=w.causal, out=t["o"], lse=t["lse"])
+        api.fwd(t["q"], t["k"], t["v"], causal=w.causal, out=t["o"], lse=t["lse"], window=_win(w))
         if events is not None:
             events["fwd"][-1][1].record()
         if with_bwd:
@@ -168,7 +180,7 @@ def _step_fn(api, t, w, with_bwd, events=None):
                                       torch.cuda.Event(enable_timing=True)))
                 events["bwd"][-1][0].record()
             api.bwd(t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], causal=w.causal,
-                    dq=t["dq"], dk=t["dk"], dv=t["dv"], workspace=t["ws"])
+                    dq=t["dq"], dk=t["dk"], dv=t["dv"], workspace=t["ws"], window=_win(w))
             if events is not None:
                 events["bwd"][-1][1].record()
     return step
@@ -189,15 +201,16 @@ def cpu_sample(w, heads: int, threads: int, rows: int | None = None, backward: b
     flops = 0.0
     for h in range(heads):
         q, k, v = (inp[n][0, :, h].double().numpy() for n in ("q", "k", "v"))
-        oracle.fwd_rows(q, k, v, w.scale, w.causal, sel)
+        oracle.fwd_rows(q, k, v, w.scale, w.causal, sel, window=w.window)
         if sel is None:
-            flops += fwd_flops(1, 1, w.N, w.d, w.causal)
+            flops += fwd_flops(1, 1, w.N, w.d, w.causal, w.window)
         else:
-            flops += sum(4.0 * ((i + 1) if w.causal else w.N) * w.d for i in sel)
+            flops += sum(4.0 * ((min(i, w.window) + 1 if w.window >= 0 else i + 1) if w.causal else w.N) * w.d
+                         for i in sel)
         if backward:
             do = inp["do"][0, :, h].double().numpy()
-            oracle.bwd_rows(q, k, v, do, w.scale, w.causal)
-            flops += bwd_flops(1, 1, w.N, w.d, w.causal)
+            oracle.bwd_rows(q, k, v, do, w.scale, w.causal, window=w.window)
+            flops += bwd_flops(1, 1, w.N, w.d, w.causal, w.window)
     dt = time.perf_counter() - t0
     return flops, dt
 
@@ -270,12 +283,12 @@ def run_ours(args, w):
     dev = torch.device("cuda", torch.cuda.current_device())
     with_bwd = with_bwd_available()
 
-    inp = make_inputs(w.B, w.H, w.N, w.d, w.seed, with_do=True, peaked=w.peaked)
+    inp = make_inputs(w.B, w.H, w.N, w.d, w.seed, with_do=True, peaked=w.peaked, H_kv=w.H_kv)
     t = {n: inp[n].to(dev) for n in ("q", "k", "v", "do")}
     t["o"] = torch.empty_like(t["q"])
     t["lse"] = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
     if with_bwd:
-        t["dq"], t["dk"], t["dv"] = (torch.empty_like(t["q"]) for _ in range(3))
+        t["dq"], t["dk"], t["dv"] = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
         t["ws"] = torch.empty(api.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
     in_bytes = sum(t[n].numel() * t[n].element_size() for n in ("q", "k", "v", "do"))
 
@@ -342,8 +355,8 @@ def run_ours(args, w):
         ms, e2e_ms, fwd_ms, bwd_ms = max_over_ranks([ms, e2e_ms, fwd_ms, bwd_ms or 0.0], dev)
         bwd_ms = bwd_ms if with_bwd else None
 
-    ff = fwd_flops(w.B, w.H, w.N, w.d, w.causal)
-    fb = bwd_flops(w.B, w.H, w.N, w.d, w.causal) if with_bwd else 0.0
+    ff = fwd_flops(w.B, w.H, w.N, w.d, w.causal, w.window)
+    fb = bwd_flops(w.B, w.H, w.N, w.d, w.causal, w.window) if with_bwd else 0.0
     step_flops = ff + fb
     value = whole_job_tflops(world, step_flops, ms)
     e2e_value = whole_job_tflops(world, step_flops, e2e_ms)
@@ -366,6 +379,7 @@ def run_ours(args, w):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "H_kv": w.H_kv or w.H, "window": w.window,
                    "parallelism": f"replicas x{world}",
                    "l2": f"not flushed: inputs {in_bytes / 1e6:.0f} MB > L2 {L2_BYTES / 1e6:.0f} MB",
                    "step": "fa_fwd + fa_bwd" if with_bwd else "fa_fwd only (backward not built)"},
@@ -400,12 +414,12 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS) + sorted(EXTRA_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    w = WORKLOADS[args.workload]
+    w = {**WORKLOADS, **EXTRA_WORKLOADS}[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

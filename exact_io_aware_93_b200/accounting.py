@@ -34,3 +34,21 @@ def bwd_bytes(B: int, H: int, N: int, d: int) -> int:
 def score_matrix_bytes(N: int, heads: int, bytes_per_score: int = 2) -> int:
     """Size of the N x N score matrix standard attention would materialise."""
     return N * N * heads * bytes_per_score
+
+
+def visible_pairs(N: int, causal: bool, window: int = -1) -> float:
+    """(query, key) pairs per head that the FLOP convention counts: N^2 (non-causal), N^2 / 2
+    (causal), and with a causal window of W keys before the query the exact count
+    sum_i min(i, W) + 1."""
+    if window < 0:
+        return N * N / 2 if causal else float(N * N)
+    w = min(window, N - 1)
+    return w * (w + 1) / 2 + (N - w) * (w + 1)
+
+
+def fwd_flops_window(B: int, H: int, N: int, d: int, causal: bool, window: int = -1) -> float:
+    return 4.0 * B * H * d * visible_pairs(N, causal, window)
+
+
+def bwd_flops_window(B: int, H: int, N: int, d: int, causal: bool, window: int = -1) -> float:
+    return 2.5 * fwd_flops_window(B, H, N, d, causal, window)

@@ -26,6 +26,13 @@ FA_STATUS = {
 }
 
 
+class FaProblem(ctypes.Structure):
+    """The ``fa_problem`` descriptor of include/fa.h."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int), ("N", ctypes.c_int),
+                ("d", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int),
+                ("window", ctypes.c_int)]
+
+
 class FAError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = int(status)
@@ -59,6 +66,13 @@ def lib() -> ctypes.CDLL:
     L.fa_selftest_wait_timeout.restype = i
     L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     L.fa_bwd_workspace_size.restype = ctypes.c_size_t
+    L.fa_fwd_ex.argtypes = [ctypes.POINTER(FaProblem), vp, vp, vp, vp, vp, vp]
+    L.fa_fwd_ex.restype = i
+    L.fa_bwd_ex.argtypes = [ctypes.POINTER(FaProblem), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                            ctypes.c_size_t, vp]
+    L.fa_bwd_ex.restype = i
+    L.fa_bwd_workspace_size_ex.argtypes = [ctypes.POINTER(FaProblem)]
+    L.fa_bwd_workspace_size_ex.restype = ctypes.c_size_t
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
                          i, i, i, i, f, i, vp]
     L.fa_bwd.restype = i
@@ -84,8 +98,9 @@ def validate_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
             raise ValueError(f"{name} must be contiguous")
     if not (q.shape[0] == k.shape[0] == v.shape[0]):
         raise ValueError(f"batch size mismatch: {q.shape[0]}, {k.shape[0]}, {v.shape[0]}")
-    if not (q.shape[2] == k.shape[2] == v.shape[2]):
-        raise ValueError(f"num heads mismatch: {q.shape[2]}, {k.shape[2]}, {v.shape[2]}")
+    if k.shape[2] != v.shape[2] or q.shape[2] % k.shape[2] != 0:
+        raise ValueError(f"num heads mismatch: {q.shape[2]}, {k.shape[2]}, {v.shape[2]} (key/value heads "
+                         "must match each other and divide the query heads)")
     if k.shape[1] != v.shape[1]:
         raise ValueError(f"key/value sequence length mismatch: {k.shape[1]}, {v.shape[1]}")
     if not (q.shape[3] == k.shape[3] == v.shape[3]):
@@ -96,22 +111,31 @@ def validate_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
         raise ValueError("q, k, v must be on the same device")
 
 
+def problem(q: torch.Tensor, k: torch.Tensor, causal: bool, scale: float | None,
+            window: int | None) -> FaProblem:
+    B, N, H, d = q.shape
+    return FaProblem(B, H, k.shape[2], N, d, 1.0 / math.sqrt(d) if scale is None else float(scale),
+                     int(bool(causal)), -1 if window is None else int(window))
+
+
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         scale: float | None = None, out: torch.Tensor | None = None,
-        lse: torch.Tensor | None = None):
-    """(O [B, N, H, d] bf16, LSE [B, H, N] fp32) of exact attention via ``fa_fwd``."""
+        lse: torch.Tensor | None = None, window: int | None = None):
+    """(O [B, N, H, d] bf16, LSE [B, H, N] fp32) of exact attention via ``fa_fwd_ex``.
+
+    k and v may have fewer heads than q (grouped-query attention); ``window`` (causal only)
+    limits query i to keys i - window .. i."""
     validate_inputs(q, k, v)
     B, N, H, d = q.shape
-    if scale is None:
-        scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                      B, H, N, d, ctypes.c_float(scale), int(bool(causal)), _stream_ptr(q))
+    p = problem(q, k, causal, scale, window)
+    st = lib().fa_fwd_ex(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                         lse.data_ptr(), _stream_ptr(q))
     if st != 0:
-        raise FAError(st, "fa_fwd")
+        raise FAError(st, "fa_fwd_ex")
     return out, lse
 
 
@@ -123,8 +147,8 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, do: torch.Tensor,
         lse: torch.Tensor, causal: bool = False, scale: float | None = None,
         dq: torch.Tensor | None = None, dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
-        workspace: torch.Tensor | None = None):
-    """(dQ, dK, dV) of L = sum(O * dO) via ``fa_bwd`` (score tiles recomputed from LSE)."""
+        workspace: torch.Tensor | None = None, window: int | None = None):
+    """(dQ, dK, dV) of L = sum(O * dO) via ``fa_bwd_ex`` (score tiles recomputed from LSE)."""
     validate_inputs(q, k, v)
     for name, t in (("o", o), ("do", do)):
         if t.shape != q.shape or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device != q.device:
@@ -132,21 +156,19 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, do: 
     B, N, H, d = q.shape
     if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
-    if scale is None:
-        scale = 1.0 / math.sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    need = bwd_workspace_size(B, H, N, d)
+    p = problem(q, k, causal, scale, window)
+    need = int(lib().fa_bwd_workspace_size_ex(ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
-    st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                      workspace.data_ptr(), ws_bytes, B, H, N, d, ctypes.c_float(scale),
-                      int(bool(causal)), _stream_ptr(q))
+    st = lib().fa_bwd_ex(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                         do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                         workspace.data_ptr(), ws_bytes, _stream_ptr(q))
     if st != 0:
-        raise FAError(st, "fa_bwd")
+        raise FAError(st, "fa_bwd_ex")
     return dq, dk, dv
 
 

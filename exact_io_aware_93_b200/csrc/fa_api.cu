@@ -71,6 +71,12 @@ fa_status current_device(DeviceInfo** out) {
   return FA_OK;
 }
 
+fa_status check_problem(const fa_problem& p) {
+  if (p.H_kv < 1 || p.H_kv > p.H || (p.H_kv >= 1 && p.H % p.H_kv != 0)) return FA_ERR_INVALID_ARG;
+  if (p.window < -1 || (p.window >= 0 && p.causal != 1)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
 fa_status check_common(int B, int H, int N, int d, float scale, int causal) {
   if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !isfinite(scale)) return FA_ERR_INVALID_ARG;
@@ -86,7 +92,7 @@ fa_status check_common(int B, int H, int N, int d, float scale, int causal) {
 
 template <int D, bool CAUSAL>
 fa_status launch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o,
-                     float* lse, int B, int H, int N, float scale, cudaStream_t stream) {
+                     float* lse, int B, int H, int H_kv, int N, int window, float scale, cudaStream_t stream) {
   auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
   const int smem = static_cast<int>(sizeof(fa::FwdSmem<D>)) + 1024;
   bool& attr = di.fwd_attr[D == 128][CAUSAL];
@@ -102,8 +108,8 @@ fa_status launch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   const long long tiles = static_cast<long long>(B) * H * ((nkb + 1) / 2);
   const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
   const float scale_log2 = scale * 1.4426950408889634f;
-  kern<<<grid, fa::kFwdThreads, smem, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, B, H, N,
-                                                 scale_log2, di.status);
+  kern<<<grid, fa::kFwdThreads, smem, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, B, H, H_kv, N,
+                                                 window, scale_log2, di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
 }
@@ -119,7 +125,8 @@ size_t bwd_ws_bytes(int B, int H, int N, int d) {
 template <int D, bool CAUSAL>
 fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& mdo, const void* o, const void* dO, const float* lse, void* dq, void* dk,
-                     void* dv, void* ws, int B, int H, int N, float scale, cudaStream_t stream) {
+                     void* dv, void* ws, int B, int H, int H_kv, int N, int window, float scale,
+                     cudaStream_t stream) {
   const int64_t rows = static_cast<int64_t>(B) * H * N;
   const int64_t prows = static_cast<int64_t>(B) * H * ((N + 127) / 128 * 128);
   float* dq_acc = static_cast<float*>(ws);
@@ -144,9 +151,10 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
     attr = true;
   }
   const int nkb = (N + 127) / 128;
-  kern<<<B * H * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, lse2, dsum, dq_acc,
-                                                        static_cast<__nv_bfloat16*>(dk),
-                                                        static_cast<__nv_bfloat16*>(dv), B, H, N, scale, di.status);
+  kern<<<B * H_kv * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, lse2, dsum, dq_acc,
+                                                           static_cast<__nv_bfloat16*>(dk),
+                                                           static_cast<__nv_bfloat16*>(dv), B, H, H_kv, N, window,
+                                                           scale, di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   fa::fa_bwd_post_kernel<D><<<ew_blocks, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), B, H, N,
                                                            scale);
@@ -212,7 +220,7 @@ fa_status noalloc_scratch(void** out) {
 
 extern "C" {
 
-int fa_abi_version(void) { return 1; }
+int fa_abi_version(void) { return 2; }
 
 const char* fa_status_string(int s) {
   switch (s) {
@@ -228,10 +236,13 @@ const char* fa_status_string(int s) {
   }
 }
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-                 float scale, int causal, void* stream) {
-  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-  fa_status st = check_common(B, H, N, d, scale, causal);
+fa_status fa_fwd_ex(const fa_problem* problem, const void* q, const void* k, const void* v, void* o, float* lse,
+                    void* stream) {
+  if (!problem || !q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  const fa_problem p = *problem;
+  fa_status st = check_common(p.B, p.H, p.N, p.d, p.scale, p.causal);
+  if (st != FA_OK) return st;
+  st = check_problem(p);
   if (st != FA_OK) return st;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGNMENT;
@@ -239,15 +250,22 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   st = current_device(&di);
   if (st != FA_OK) return st;
   CUtensorMap mq, mk, mv;
-  if (!fa::make_bshd_map(&mq, q, B, N, H, d, 128) || !fa::make_bshd_map(&mk, k, B, N, H, d, 128) ||
-      !fa::make_bshd_map(&mv, v, B, N, H, d, 128))
+  if (!fa::make_bshd_map(&mq, q, p.B, p.N, p.H, p.d, 128) || !fa::make_bshd_map(&mk, k, p.B, p.N, p.H_kv, p.d, 128) ||
+      !fa::make_bshd_map(&mv, v, p.B, p.N, p.H_kv, p.d, 128))
     return FA_ERR_LAUNCH;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 128)
-    return causal ? launch_fwd<128, true>(*di, mq, mk, mv, o, lse, B, H, N, scale, s)
-                  : launch_fwd<128, false>(*di, mq, mk, mv, o, lse, B, H, N, scale, s);
-  return causal ? launch_fwd<64, true>(*di, mq, mk, mv, o, lse, B, H, N, scale, s)
-                : launch_fwd<64, false>(*di, mq, mk, mv, o, lse, B, H, N, scale, s);
+  const int w = p.window;
+  if (p.d == 128)
+    return p.causal ? launch_fwd<128, true>(*di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s)
+                    : launch_fwd<128, false>(*di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s);
+  return p.causal ? launch_fwd<64, true>(*di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s)
+                  : launch_fwd<64, false>(*di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s);
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, void* stream) {
+  const fa_problem p{B, H, H, N, d, scale, causal, -1};
+  return fa_fwd_ex(&p, q, k, v, o, lse, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -255,11 +273,21 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return bwd_ws_bytes(B, H, N, d);
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
-                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
-                 float scale, int causal, void* stream) {
-  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+size_t fa_bwd_workspace_size_ex(const fa_problem* p) {
+  if (!p) return 0;
+  return fa_bwd_workspace_size(p->B, p->H, p->N, p->d);
+}
+
+fa_status fa_bwd_ex(const fa_problem* problem, const void* q, const void* k, const void* v, const void* o,
+                    const void* dO, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (!problem || !q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  const fa_problem p = *problem;
+  const int B = p.B, H = p.H, H_kv = p.H_kv, N = p.N, d = p.d, causal = p.causal, window = p.window;
+  const float scale = p.scale;
   fa_status st = check_common(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  st = check_problem(p);
   if (st != FA_OK) return st;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
       !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
@@ -271,15 +299,26 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   st = current_device(&di);
   if (st != FA_OK) return st;
   CUtensorMap mq, mk, mv, mdo;
-  if (!fa::make_bshd_map(&mq, q, B, N, H, d, 128) || !fa::make_bshd_map(&mk, k, B, N, H, d, 128) ||
-      !fa::make_bshd_map(&mv, v, B, N, H, d, 128) || !fa::make_bshd_map(&mdo, dO, B, N, H, d, 128))
+  if (!fa::make_bshd_map(&mq, q, B, N, H, d, 128) || !fa::make_bshd_map(&mk, k, B, N, H_kv, d, 128) ||
+      !fa::make_bshd_map(&mv, v, B, N, H_kv, d, 128) || !fa::make_bshd_map(&mdo, dO, B, N, H, d, 128))
     return FA_ERR_LAUNCH;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 128)
-    return causal ? launch_bwd<128, true>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s)
-                  : launch_bwd<128, false>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s);
-  return causal ? launch_bwd<64, true>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s)
-                : launch_bwd<64, false>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, N, scale, s);
+    return causal ? launch_bwd<128, true>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, H_kv, N,
+                                          window, scale, s)
+                  : launch_bwd<128, false>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, H_kv, N,
+                                           window, scale, s);
+  return causal ? launch_bwd<64, true>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, H_kv, N,
+                                       window, scale, s)
+                : launch_bwd<64, false>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, H_kv, N,
+                                        window, scale, s);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                 float scale, int causal, void* stream) {
+  const fa_problem p{B, H, H, N, d, scale, causal, -1};
+  return fa_bwd_ex(&p, q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,

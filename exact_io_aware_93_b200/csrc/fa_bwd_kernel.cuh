@@ -11,8 +11,10 @@
 // Three kernels, one stream:
 //   fa_bwd_pre  : D_i and LSE_i * log2 e (fp32, padded per head to whole 128-row blocks) and
 //                 zeroing of the fp32 dQ accumulator (memory bound)
-//   fa_bwd_main : one CTA per (batch, head, 128-key block j), head-major; K_j and V_j stay in shared
-//                 memory while 128-query blocks i (i >= j when causal) stream through:
+//   fa_bwd_main : one CTA per (batch, key/value head, 128-key block j), head-major; K_j and
+//                 V_j stay in shared memory while, for every query head of the group that
+//                 shares the key/value head, the 128-query blocks i that see block j
+//                 (i >= j when causal, within the window when there is one) stream through:
 //                   S^T  = K_j Q_i^T        (tcgen05, both operands in shared memory)
 //                   dP^T = V_j dO_i^T
 //                   P^T  = 2^(S^T * scale * log2 e - LSE_i * log2 e)   (one thread per key)
@@ -24,7 +26,8 @@
 //                                           so that tensor-memory lanes are head-dim columns
 //                 and a drain warpgroup copies each dQ_i tile out of tensor memory, frees it,
 //                 and adds it into the fp32 accumulator with reductions that cover whole
-//                 128-byte lines; dK_j, dV_j are written once at the end.
+//                 128-byte lines; dK_j, dV_j accumulate over the whole group in tensor
+//                 memory and are written once at the end.
 //   Per query block the MMA warp issues dP, then (once P is ready) dV and the next block's
 //   S, then (once dS is ready) dK and dQ, so the tensor core works while the key-row
 //   warpgroups compute dS and while the drain empties the previous dQ tile.
@@ -172,12 +175,13 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 }
 
 // P^T for 32 queries of one key row: p = 2^(s * sl - lse2), zero where masked
-// (MASKED: key beyond the sequence, or query index below qlim on the diagonal block);
+// (MASKED: key beyond the sequence, query index below qlim on the diagonal block, or above
+// qhi past the end of a sliding window);
 // returns the 16 bf16 pairs.  One branch per chunk instead of one per element keeps the
 // unrolled loop a single basic block the compiler can interleave.
 template <bool MASKED>
 __device__ __forceinline__ void bwd_p_chunk(const uint32_t (&sv)[32], const float* lse2, float2 sl2, int q0,
-                                            bool key_ok, int qlim, uint32_t* pk) {
+                                            bool key_ok, int qlim, int qhi, uint32_t* pk) {
   float4 l4[8];
 #pragma unroll
   for (int y = 0; y < 8; ++y) l4[y] = reinterpret_cast<const float4*>(lse2)[y];
@@ -191,10 +195,10 @@ __device__ __forceinline__ void bwd_p_chunk(const uint32_t (&sv)[32], const floa
     float p0 = ex2_approx(a.x), p1 = ex2_approx(a.y), p2 = ex2_approx(b.x), p3 = ex2_approx(b.y);
     if (MASKED) {
       const int ql = q0 + x;
-      p0 = (key_ok && ql >= qlim) ? p0 : 0.f;
-      p1 = (key_ok && ql + 1 >= qlim) ? p1 : 0.f;
-      p2 = (key_ok && ql + 2 >= qlim) ? p2 : 0.f;
-      p3 = (key_ok && ql + 3 >= qlim) ? p3 : 0.f;
+      p0 = (key_ok && ql >= qlim && ql <= qhi) ? p0 : 0.f;
+      p1 = (key_ok && ql + 1 >= qlim && ql + 1 <= qhi) ? p1 : 0.f;
+      p2 = (key_ok && ql + 2 >= qlim && ql + 2 <= qhi) ? p2 : 0.f;
+      p3 = (key_ok && ql + 3 >= qlim && ql + 3 <= qhi) ? p3 : 0.f;
     }
     pk[x / 2] = pack_bf16x2(p0, p1);
     pk[x / 2 + 1] = pack_bf16x2(p2, p3);
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                        const float* __restrict__ lse2g, const float* __restrict__ dsum,
                        float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                       int B, int H, int N, float scale, int* status) {
+                       int B, int H, int H_kv, int N, int window, float scale, int* status) {
   using Cfg = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {  // the layout relies on a 1 KB aligned base
@@ -219,16 +223,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int nkb = (N + 127) / 128;
-  const int BH = B * H;
+  const int group = H / H_kv;  // query heads sharing this key/value head
   // Head-major order: the CTAs resident at any time cover only a few heads, so their dQ
   // accumulator rows and Q/dO tiles stay in L2.  Within a head, key blocks go heaviest
   // first (with causal masking block j meets nkb - j query blocks), so the grid ends on
   // the lightest blocks.
-  const int bh = blockIdx.x / nkb;
+  const int bhkv = blockIdx.x / nkb;
   const int j = blockIdx.x % nkb;
-  const int b = bh / H, h = bh % H;
+  const int b = bhkv / H_kv, hkv = bhkv % H_kv;
+  // query blocks that see key block j: i >= j when causal, and with a window only those
+  // whose first query is within `window` of the block's last key
   const int i0 = CAUSAL ? j : 0;
-  const int ni = nkb - i0;
+  int i1 = nkb;
+  if (window >= 0) {
+    const int last = (j * 128 + 127 + window) / 128 + 1;
+    i1 = last < nkb ? last : nkb;
+  }
+  const int nper = i1 - i0;     // query blocks per query head
+  const int ni = group * nper;  // iterations: every query head of the group, every block
 
   if (threadIdx.x == 0) {
     sm.abort_flag = 0;
@@ -270,8 +282,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(&sm.kv_full, 2 * Cfg::kTileBytes);
       for (int c = 0; c < Cfg::kChunks; ++c) {
-        tma_load_4d(sm.k + c * Cfg::kChunkBytes, &tm_k, &sm.kv_full, c * 64, h, j * 128, b);
-        tma_load_4d(sm.v + c * Cfg::kChunkBytes, &tm_v, &sm.kv_full, c * 64, h, j * 128, b);
+        tma_load_4d(sm.k + c * Cfg::kChunkBytes, &tm_k, &sm.kv_full, c * 64, hkv, j * 128, b);
+        tma_load_4d(sm.v + c * Cfg::kChunkBytes, &tm_v, &sm.kv_full, c * 64, hkv, j * 128, b);
       }
     }
     const int npad = nkb * 128;
@@ -279,7 +291,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (int idx = 0; idx < ni; ++idx) {
       const int st = idx & 1;
-      const int i = i0 + idx;
+      const int i = i0 + idx % nper;
+      const int h = hkv * group + idx / nper;
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.qd_empty[st], ((idx >> 1) & 1) ^ 1, wc));
       if (!ok) break;
       if (lane == 0) {
@@ -289,7 +302,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_4d(sm.q[st] + c * Cfg::kChunkBytes, &tm_q, &sm.qd_full[st], c * 64, h, i * 128, b);
           tma_load_4d(sm.dO[st] + c * Cfg::kChunkBytes, &tm_do, &sm.qd_full[st], c * 64, h, i * 128, b);
         }
-        const int64_t ridx = static_cast<int64_t>(bh) * npad + i * 128;
+        const int64_t ridx = (static_cast<int64_t>(b) * H + h) * npad + i * 128;
         bulk_load(sm.lse2[st], lse2g + ridx, 512, &sm.qd_full[st]);
         bulk_load(sm.dd[st], dsum + ridx, 512, &sm.qd_full[st]);
       }
@@ -398,15 +411,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (int idx = 0; idx < ni && ok; ++idx) {
       const int st = idx & 1;
-      const int i = i0 + idx;
+      const int i = i0 + idx % nper;
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.qd_full[st], (idx >> 1) & 1, wc));
       ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.s_full, idx & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      // valid (query q, key k): k < N, and k <= q when causal; q >= N has LSE = +inf -> P = 0
+      // valid (query q, key k): k < N, k <= q when causal, q <= k + window with a window;
+      // q >= N has LSE = +inf -> P = 0
       const bool key_ok = kg < N;
-      const int qlim = (CAUSAL && i == j) ? r - 64 * g : 0;  // diagonal block: query >= key
-      const bool masked = __any_sync(0xffffffffu, !key_ok || qlim > 0);
+      const int qbase = i * 128 + 64 * g;                            // first query of this half
+      const int qlim = (CAUSAL && i == j) ? r - 64 * g : 0;          // diagonal block: query >= key
+      const int qhi = window >= 0 ? kg + window - qbase : 1 << 30;   // query <= key + window
+      const bool masked = __any_sync(0xffffffffu, !key_ok || qlim > 0 || qhi < 63);
       const float* lse2 = sm.lse2[st] + 64 * g;
       const float* dd = sm.dd[st] + 64 * g;
       // bf16 P^T of this key row for the warpgroup's 64 queries, packed in pairs; dS uses the
@@ -419,9 +435,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_wait_ld();
         uint32_t* pk = pk_all + 16 * c;
         if (masked)
-          bwd_p_chunk<true>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, pk);
+          bwd_p_chunk<true>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, qhi, pk);
         else
-          bwd_p_chunk<false>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, pk);
+          bwd_p_chunk<false>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, qhi, pk);
         tmem_st16(tS + c * 16, pk);  // columns already read
       }
       tmem_wait_st();
@@ -472,7 +488,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const uint32_t tAcc = tbase + (g == 0 ? Cfg::kColDV : Cfg::kColDK) + lane_off;
       const float mul = g == 0 ? 1.0f : scale;
-      __nv_bfloat16* dst = (g == 0 ? dv : dk) + ((static_cast<int64_t>(b) * N + kg) * H + h) * D;
+      __nv_bfloat16* dst = (g == 0 ? dv : dk) + ((static_cast<int64_t>(b) * N + kg) * H_kv + hkv) * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t a[32];
@@ -502,7 +518,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, idx & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      const int q0 = (i0 + idx) * 128;
+      const int q0 = (i0 + idx % nper) * 128;
+      const int64_t bh = static_cast<int64_t>(b) * H + hkv * group + idx / nper;  // query head row
       if constexpr (D == 128) {
         // lane r holds column r of dQ_i for the 128 queries; a warp's reduction for one query
         // covers 32 consecutive columns = one 128-byte line
@@ -515,13 +532,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         mbar_arrive(&sm.dq_free);  // the dP columns may be overwritten from here on
         const int qn = min(128, N - q0);
-        float* dst = dq_acc + (static_cast<int64_t>(bh) * N + q0) * D + r;
+        float* dst = dq_acc + (bh * N + q0) * D + r;
 #pragma unroll
         for (int q = 0; q < 128; ++q)
           if (q < qn) red_add(dst + static_cast<int64_t>(q) * D, __uint_as_float(a[q]));
       } else {
         const int qg = q0 + r;
-        float* dst = dq_acc + (static_cast<int64_t>(bh) * N + qg) * D;
+        float* dst = dq_acc + (bh * N + qg) * D;
         uint32_t a[D];
 #pragma unroll
         for (int c = 0; c < D; c += 32) tmem_ld32(tQ + c, a + c);

@@ -1,8 +1,11 @@
 // fa_fwd_kernel.cuh -- fused exact-attention forward for sm_100a.
 //
 // One persistent CTA per SM walks a list of work tiles.  A tile is one
-// (batch, head) and a PAIR of 128-row query blocks; the pair shares one stream
-// of 128-key K/V tiles ("Flash Attention Explained", institutepm.com, "Tile the
+// (batch, query head) and a PAIR of 128-row query blocks; the pair shares one stream
+// of 128-key K/V tiles of its key/value head (H / H_kv query heads share one
+// key/value head: grouped-query attention, "Flash Attention Explained", "Grouped
+// Query Attention"), optionally limited to a causal sliding window (same page,
+// "Sliding Window Attention") ("Flash Attention Explained", institutepm.com, "Tile the
 // input" / "Fuse into one kernel"; FlashAttention-2's partitioning over the
 // sequence dimension, same page, "Flash Attention 1, 2, and 3").
 //
@@ -107,11 +110,22 @@ __device__ __forceinline__ FwdTile fwd_decode(int t, int BH, int H, int npairs) 
   return ti;
 }
 
-// Number of K/V tiles query block qb visits (0 if the block lies past the sequence).
+// Key blocks [lo, hi) that query block qb visits (empty past the sequence).  With causal
+// masking the last is the diagonal block; with a sliding window of `window` keys before
+// the query, the first is the block holding key qb*128 - window.
+struct KvRange {
+  int lo, hi;
+};
 template <bool CAUSAL>
-__device__ __forceinline__ int fwd_nblocks(int qb, int nkb) {
-  if (qb >= nkb) return 0;
-  return CAUSAL ? qb + 1 : nkb;
+__device__ __forceinline__ KvRange fwd_range(int qb, int nkb, int window) {
+  KvRange r{0, 0};
+  if (qb >= nkb) return r;
+  r.hi = CAUSAL ? qb + 1 : nkb;
+  if (window >= 0) {
+    const int first_key = qb * kBM - window;
+    r.lo = first_key > 0 ? first_key / kBN : 0;
+  }
+  return r;
 }
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int* status) {
@@ -166,7 +180,8 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-                  float* __restrict__ lse, int B, int H, int N, float scale_log2, int* status) {
+                  float* __restrict__ lse, int B, int H, int H_kv, int N, int window, float scale_log2,
+                  int* status) {
   using Cfg = FwdCfg<D>;
   constexpr int NS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -178,6 +193,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int npairs = (nkb + 1) / 2;
   const int BH = B * H;
   const int T = BH * npairs;
+  const int group = H / H_kv;  // query heads per key/value head
 
   if (threadIdx.x == 0) {
     sm.abort_flag = 0;
@@ -223,9 +239,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int t = snake_tile(blockIdx.x, k, gridDim.x);
         if (t >= T) break;
         const FwdTile ti = fwd_decode(t, BH, H, npairs);
-        const int n[2] = {fwd_nblocks<CAUSAL>(ti.qb0, nkb), fwd_nblocks<CAUSAL>(ti.qb0 + 1, nkb)};
+        const KvRange rg[2] = {fwd_range<CAUSAL>(ti.qb0, nkb, window), fwd_range<CAUSAL>(ti.qb0 + 1, nkb, window)};
+        const int hkv = ti.h / group;
         for (int i = 0; i < 2 && ok; ++i) {
-          if (n[i] == 0) continue;
+          if (rg[i].hi == rg[i].lo) continue;
           ok = mbar_wait(&sm.q_empty[i], (qcnt[i] & 1) ^ 1, wc);
           if (!ok) break;
           mbar_arrive_expect_tx(&sm.q_full[i], Cfg::kTileBytes);
@@ -234,8 +251,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         ti.b);
           ++qcnt[i];
         }
-        const int nkv = n[0] > n[1] ? n[0] : n[1];
-        for (int j = 0; j < nkv && ok; ++j) {
+        // K/V stream: the union of both blocks' ranges (block 1's range starts and ends later)
+        const int jlo = rg[0].lo;
+        const int jhi = rg[1].hi > rg[0].hi ? rg[1].hi : rg[0].hi;
+        for (int j = jlo; j < jhi && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv, ++it) {
             const int s = it % NS;
             ok = mbar_wait(&sm.kv_empty[s], ((it / NS) & 1) ^ 1, wc);
@@ -243,7 +262,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_arrive_expect_tx(&sm.kv_full[s], Cfg::kTileBytes);
             const CUtensorMap* m = kv ? &tm_v : &tm_k;
             for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_4d(sm.kv[s] + c * Cfg::kChunkBytes, m, &sm.kv_full[s], c * 64, ti.h, j * kBN, ti.b);
+              tma_load_4d(sm.kv[s] + c * Cfg::kChunkBytes, m, &sm.kv_full[s], c * 64, hkv, j * kBN, ti.b);
           }
         }
       }
@@ -293,48 +312,51 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int t = snake_tile(blockIdx.x, k, gridDim.x);
         if (t >= T) break;
         const FwdTile ti = fwd_decode(t, BH, H, npairs);
-        const int n[2] = {fwd_nblocks<CAUSAL>(ti.qb0, nkb), fwd_nblocks<CAUSAL>(ti.qb0 + 1, nkb)};
-        const int nkv = n[0] > n[1] ? n[0] : n[1];
+        const KvRange rg[2] = {fwd_range<CAUSAL>(ti.qb0, nkb, window), fwd_range<CAUSAL>(ti.qb0 + 1, nkb, window)};
+        const int jlo = rg[0].lo;
+        const int jhi = rg[1].hi > rg[0].hi ? rg[1].hi : rg[0].hi;
+        auto in = [&](int i, int j) { return j >= rg[i].lo && j < rg[i].hi; };
         for (int i = 0; i < 2 && ok; ++i)
-          if (n[i] > 0) ok = mbar_wait(&sm.q_full[i], qcnt[i] & 1, wc);
+          if (rg[i].hi > rg[i].lo) ok = mbar_wait(&sm.q_full[i], qcnt[i] & 1, wc);
         if (!ok) break;
-        // prologue: S_i(0)
+        // prologue: S_i for the first key block
         const int sk0 = it % NS;
         ok = mbar_wait(&sm.kv_full[sk0], (it / NS) & 1, wc);
         if (!ok) break;
         ++it;
         tc_fence_after();
         for (int i = 0; i < 2; ++i) {
-          if (n[i] == 0) continue;
+          if (!in(i, jlo)) continue;
           issue_s(i, sk0);
           umma_commit(&sm.s_full[i]);
-          if (n[i] == 1) umma_commit(&sm.q_empty[i]);
+          if (rg[i].hi == jlo + 1) umma_commit(&sm.q_empty[i]);
         }
         umma_commit(&sm.kv_empty[sk0]);
-        for (int j = 0; j < nkv && ok; ++j) {
+        for (int j = jlo; j < jhi && ok; ++j) {
           const int sv = it % NS;
           ok = mbar_wait(&sm.kv_full[sv], (it / NS) & 1, wc);
           if (!ok) break;
           ++it;
           int skn = -1;
-          if (j + 1 < nkv) {
+          if (j + 1 < jhi) {
             skn = it % NS;
             ok = mbar_wait(&sm.kv_full[skn], (it / NS) & 1, wc);
             if (!ok) break;
             ++it;
           }
           for (int i = 0; i < 2 && ok; ++i) {
-            if (j >= n[i]) continue;
-            ok = mbar_wait(&sm.p_full[i], pcnt[i] & 1, wc);
-            if (!ok) break;
-            ++pcnt[i];
-            tc_fence_after();
-            issue_pv(i, sv, j > 0);
-            if (j + 1 == n[i]) umma_commit(&sm.o_done[i]);
-            if (j + 1 < n[i]) {
+            if (in(i, j)) {
+              ok = mbar_wait(&sm.p_full[i], pcnt[i] & 1, wc);
+              if (!ok) break;
+              ++pcnt[i];
+              tc_fence_after();
+              issue_pv(i, sv, j > rg[i].lo);
+              if (j + 1 == rg[i].hi) umma_commit(&sm.o_done[i]);
+            }
+            if (in(i, j + 1)) {
               issue_s(i, skn);
               umma_commit(&sm.s_full[i]);
-              if (j + 2 == n[i]) umma_commit(&sm.q_empty[i]);
+              if (j + 2 == rg[i].hi) umma_commit(&sm.q_empty[i]);
             }
           }
           if (!ok) break;
@@ -342,7 +364,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (skn >= 0) umma_commit(&sm.kv_empty[skn]);
         }
         for (int i = 0; i < 2; ++i)
-          if (n[i] > 0) ++qcnt[i];
+          if (rg[i].hi > rg[i].lo) ++qcnt[i];
       }
       // Wait for every MMA issued to finish before the columns are freed.
       umma_commit(&sm.mma_drain);
@@ -366,13 +388,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (t >= T) break;
       const FwdTile ti = fwd_decode(t, BH, H, npairs);
       const int qb = ti.qb0 + g;
-      const int n = fwd_nblocks<CAUSAL>(qb, nkb);
-      if (n == 0) continue;
+      const KvRange rg = fwd_range<CAUSAL>(qb, nkb, window);
+      if (rg.hi == rg.lo) continue;
       const int row = qb * kBM + r;
       float m_ref = -INFINITY;
       float l = 0.f;    // sum of 2^(x - m) in fp32: the log-sum-exp
       float lr = 0.f;   // sum of the same weights rounded to bf16: normalises O
-      for (int j = 0; j < n; ++j) {
+      for (int j = rg.lo; j < rg.hi; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[g], scnt & 1, wc));
         if (!ok) break;
         ++scnt;
@@ -384,13 +406,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tmem_ld32(tS + 96, s + 96);
         tmem_wait_ld();
         const int k0 = j * kBN;
-        const bool masked = (j == n - 1) && (CAUSAL || (N % kBN) != 0);
+        // masking: the diagonal / last tile (causal, or keys past N), and with a window the
+        // tiles that start before some row's first visible key
+        const bool edge = window >= 0 && k0 < qb * kBM + kBM - 1 - window;
+        const bool masked = ((j == rg.hi - 1) && (CAUSAL || (N % kBN) != 0)) || edge;
         if (masked) {
           int lim = N - 1 - k0;                    // last valid key column of this tile
-          if (CAUSAL) lim = min(lim, row - k0);    // diagonal tile: key <= query
+          if (CAUSAL) lim = min(lim, row - k0);    // key <= query
+          const int first = window >= 0 ? row - window - k0 : 0;  // key >= query - window
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
-            if (c > lim) s[c] = __float_as_uint(-INFINITY);
+            if (c > lim || c < first) s[c] = __float_as_uint(-INFINITY);
         }
         // row maximum: 8 independent chains of three-input max, then combine
         float mx8[8];
@@ -412,7 +438,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             lr *= alpha;
             m_ref = m_new;
           }
-          if (j > 0) {
+          if (j > rg.lo) {
             // PV(j-1) is complete: the commit that signalled S(j) covers it.
 #pragma unroll 1
             for (int c = 0; c < D; c += 32) {
@@ -427,11 +453,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
         uint32_t p[kBN / 2];
+        // a row that has seen no visible key yet (window edge) keeps m = -inf; use 0 as its
+        // reference so that 2^(-inf - m) stays 0 instead of NaN
+        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
         // masked tiles hold -inf scores: they stay on the MUFU path (2^-inf = 0 exactly)
         if (masked)
-          softmax_row<false>(s, p, scale_log2, m_ref, l, lr);
+          softmax_row<false>(s, p, scale_log2, m_use, l, lr);
         else
-          softmax_row<true>(s, p, scale_log2, m_ref, l, lr);
+          softmax_row<true>(s, p, scale_log2, m_use, l, lr);
         tmem_st32(tS + 0, p);
         tmem_st32(tS + 32, p + 32);
         tmem_wait_st();

@@ -37,6 +37,8 @@ class Workload:
     seed: int
     backward: bool = False
     peaked: bool = False
+    H_kv: int | None = None          # key/value heads (None: same as H)
+    window: int = -1                 # causal sliding window (-1: none)
     # forward rows checked per head (None = every row)
     rows_per_head: int | None = None
     # backward: heads checked in full, plus (extra_heads x extra_rows_per_head) sampled rows
@@ -72,21 +74,38 @@ WORKLOADS = {
 }
 
 
+# Workloads of the rows beyond the five configurations: grouped-query heads and a causal
+# sliding window, at the shapes of common long-context models.
+EXTRA_WORKLOADS = {
+    w.name: w
+    for w in [
+        Workload("gqa_causal_fwdbwd_b2_h32_hkv8_n8192_d128", 2, 32, 8192, 128, True, 1101,
+                 backward=True, H_kv=8,
+                 notes="4 query heads per key/value head, causal forward + backward"),
+        Workload("window4096_causal_fwdbwd_b1_h32_hkv8_n32768_d128", 1, 32, 32768, 128, True, 1102,
+                 backward=True, H_kv=8, window=4096,
+                 notes="grouped heads + causal sliding window of 4096 keys, forward + backward"),
+    ]
+}
+
+
 def peaked_positions(N: int, gen: torch.Generator) -> torch.Tensor:
     """floor(N/100) distinct sequence positions, drawn by a seeded permutation."""
     return torch.randperm(N, generator=gen)[: N // 100]
 
 
 def make_inputs(B: int, H: int, N: int, d: int, seed: int, *, with_do: bool = False,
-                peaked: bool = False) -> dict[str, torch.Tensor]:
-    """CPU bf16 tensors ``q, k, v`` (and ``do``) of shape [B, N, H, d]."""
+                peaked: bool = False, H_kv: int | None = None) -> dict[str, torch.Tensor]:
+    """CPU bf16 tensors ``q`` (and ``do``) of shape [B, N, H, d] and ``k, v`` of shape
+    [B, N, H_kv, d] (H_kv defaults to H)."""
     gen = torch.Generator(device="cpu")
     gen.manual_seed(int(seed))
-    shape = (B, N, H, d)
+    hkv = H if H_kv is None else int(H_kv)
     out = {}
     names = ["q", "k", "v"] + (["do"] if with_do else [])
     for name in names:
-        out[name] = torch.randn(shape, generator=gen, dtype=torch.float32)
+        heads = hkv if name in ("k", "v") else H
+        out[name] = torch.randn((B, N, heads, d), generator=gen, dtype=torch.float32)
     if peaked:
         pos = peaked_positions(N, gen)
         out["k"][:, pos] *= 3.0
@@ -97,7 +116,7 @@ def make_inputs(B: int, H: int, N: int, d: int, seed: int, *, with_do: bool = Fa
 
 
 def make_workload_inputs(w: Workload) -> dict[str, torch.Tensor]:
-    return make_inputs(w.B, w.H, w.N, w.d, w.seed, with_do=w.backward, peaked=w.peaked)
+    return make_inputs(w.B, w.H, w.N, w.d, w.seed, with_do=w.backward, peaked=w.peaked, H_kv=w.H_kv)
 
 
 def sample_rows(N: int, count: int | None, seed: int) -> torch.Tensor:

@@ -56,8 +56,34 @@ typedef enum {
   FA_ERR_WORKSPACE = 7    /* workspace pointer NULL or smaller than the required size */
 } fa_status;
 
-/* Library ABI version (this header: 1). */
+/* Library ABI version (this header: 2). */
 int fa_abi_version(void);
+
+/*
+ * Problem description for the _ex entry points.
+ *   B, N, d      : batch, sequence length (queries and keys), head dimension (64 or 128)
+ *   H            : query heads
+ *   H_kv         : key/value heads, 1 <= H_kv <= H and H % H_kv == 0; query head h uses
+ *                  key/value head h / (H / H_kv) -- grouped-query attention, and multi-query
+ *                  attention for H_kv = 1 ("Flash Attention Explained", institutepm.com,
+ *                  "Grouped Query Attention": orthogonal to Flash Attention).  H_kv = H is
+ *                  ordinary multi-head attention.
+ *   scale        : softmax scale (> 0, finite)
+ *   causal       : 0 or 1
+ *   window       : -1 for none; >= 0 (causal only) limits query i to keys i - window .. i,
+ *                  sliding-window attention (same page, "Sliding Window Attention").
+ * Tensors: q, o, dO, dq are [B, N, H, d]; k, v, dk, dv are [B, N, H_kv, d]; lse is [B, H, N].
+ */
+typedef struct fa_problem {
+  int B;
+  int H;
+  int H_kv;
+  int N;
+  int d;
+  float scale;
+  int causal;
+  int window;
+} fa_problem;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);
@@ -73,6 +99,12 @@ const char* fa_status_string(int status);
  */
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  float scale, int causal, void* stream);
+
+/* fa_fwd for a general problem (grouped-query heads, sliding window).  Errors as fa_fwd,
+ * plus FA_ERR_INVALID_ARG for a NULL problem, H_kv not dividing H, window < -1, or a
+ * window without causal masking. */
+fa_status fa_fwd_ex(const fa_problem* problem, const void* q, const void* k, const void* v, void* o,
+                    float* lse, void* stream);
 
 /*
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ accumulator
@@ -99,6 +131,17 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
                  float scale, int causal, void* stream);
+
+/* Workspace bytes fa_bwd_ex needs for a problem (same as fa_bwd_workspace_size for its
+ * B, H, N, d: the accumulator and statistics are per query head). 0 for a NULL problem. */
+size_t fa_bwd_workspace_size_ex(const fa_problem* problem);
+
+/* fa_bwd for a general problem: k, v, dk, dv are [B, N, H_kv, d]; dK and dV of a shared
+ * key/value head accumulate the contributions of all H / H_kv query heads that use it.
+ * Errors as fa_bwd, plus those of fa_fwd_ex for the problem. */
+fa_status fa_bwd_ex(const fa_problem* problem, const void* q, const void* k, const void* v, const void* o,
+                    const void* dO, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                    size_t workspace_bytes, void* stream);
 
 /*
  * fa_bwd without a workspace argument, for callers that cannot allocate device memory:

@@ -46,7 +46,7 @@ def test_status_strings(lib):
     assert lib.fa_status_string(0) == b"FA_OK"
     assert lib.fa_status_string(6) == b"FA_ERR_TIMEOUT"
     assert lib.fa_status_string(99) == b"FA_ERR_UNKNOWN"
-    assert lib.fa_abi_version() == 1
+    assert lib.fa_abi_version() == 2
 
 
 def _fwd(lib, q=0x10000, k=0x10000, v=0x10000, o=0x10000, lse=0x10000, B=1, H=1, N=16, d=64,
@@ -112,3 +112,28 @@ def test_selftest_validation_without_gpu(lib):
     lib.fa_selftest_wait_timeout.restype = ctypes.c_int
     assert lib.fa_selftest_wait_timeout(0, None) == 1
     assert lib.fa_selftest_wait_timeout(5_000_000, None) == 1
+
+
+def test_ex_validation_codes(lib):
+    from exact_io_aware_93_b200.api import FaProblem
+    vp = ctypes.c_void_p
+    lib.fa_fwd_ex.argtypes = [ctypes.POINTER(FaProblem), vp, vp, vp, vp, vp, vp]
+    lib.fa_fwd_ex.restype = ctypes.c_int
+    lib.fa_bwd_workspace_size_ex.argtypes = [ctypes.POINTER(FaProblem)]
+    lib.fa_bwd_workspace_size_ex.restype = ctypes.c_size_t
+    P = 0x10000
+
+    def fwd(**kw):
+        base = dict(B=1, H=4, H_kv=2, N=64, d=64, scale=0.125, causal=1, window=-1)
+        base.update(kw)
+        p = FaProblem(**base)
+        return lib.fa_fwd_ex(ctypes.byref(p), vp(P), vp(P), vp(P), vp(P), vp(P), None)
+    assert lib.fa_fwd_ex(None, vp(P), vp(P), vp(P), vp(P), vp(P), None) == 1
+    assert fwd(H_kv=3) == 1          # does not divide H
+    assert fwd(H_kv=0) == 1
+    assert fwd(H_kv=8) == 1          # more key/value heads than query heads
+    assert fwd(window=-2) == 1
+    assert fwd(window=5, causal=0) == 1
+    assert fwd(d=96) == 2
+    p = FaProblem(2, 4, 1, 100, 128, 0.1, 1, 16)
+    assert lib.fa_bwd_workspace_size_ex(ctypes.byref(p)) == 4 * 2 * 4 * (100 * 128 + 2 * 128)
