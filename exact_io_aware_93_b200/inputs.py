@@ -89,6 +89,81 @@ EXTRA_WORKLOADS = {
 }
 
 
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Decoding: N_q new queries per sequence against a key/value cache of capacity N_kv."""
+    name: str
+    B: int
+    H: int
+    H_kv: int
+    N_q: int
+    N_kv: int
+    d: int
+    causal: bool
+    seed: int
+    lengths: str = "mixed"           # "full": every sequence N_kv long; "mixed": see make_decode_inputs
+    window: int = -1
+    checked_heads: int = 8           # (b, h) pairs checked against the oracle at full size
+    notes: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(self.d) ** 0.5
+
+
+# Decoding at the head counts of an 8B-class model with grouped key/value heads: one new
+# token per sequence, 16 sequences whose cached lengths are spread over [N_kv / 2, N_kv].
+DECODE_WORKLOADS = {
+    w.name: w
+    for w in [
+        DecodeWorkload("decode_b16_h32_hkv8_nq1_nkv32768_d128", 16, 32, 8, 1, 32768, 128, True, 1201,
+                       notes="one new token per sequence, cache lengths spread over [16384, 32768]"),
+    ]
+}
+
+
+def make_decode_inputs(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int, seed: int, *,
+                       lengths="mixed", tail_nan: bool = False) -> dict[str, torch.Tensor]:
+    """CPU tensors for decoding: ``q`` bf16 [B, N_q, H, d], ``k``/``v`` bf16 [B, N_kv, H_kv, d]
+    (the cache) and ``seqlens`` int32 [B].
+
+    Recipe: a ``torch.Generator('cpu')`` seeded with ``seed`` draws fp32 standard normals
+    for q, k, v in that order, rounded to bf16; then the lengths: ``"full"`` gives N_kv
+    for every sequence, ``"mixed"`` draws each uniformly from [N_kv // 2, N_kv] with the
+    same generator, and a sequence of ints is taken as given.  With ``tail_nan`` the cache
+    positions past each length are overwritten with NaN (stale cache slots must not matter).
+    """
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    out = {
+        "q": torch.randn((B, N_q, H, d), generator=gen, dtype=torch.float32).to(torch.bfloat16),
+        "k": torch.randn((B, N_kv, H_kv, d), generator=gen, dtype=torch.float32).to(torch.bfloat16),
+        "v": torch.randn((B, N_kv, H_kv, d), generator=gen, dtype=torch.float32).to(torch.bfloat16),
+    }
+    if isinstance(lengths, str):
+        if lengths == "full":
+            lens = torch.full((B,), N_kv, dtype=torch.int32)
+        elif lengths == "mixed":
+            lens = torch.randint(N_kv // 2, N_kv + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
+        else:
+            raise ValueError(f"unknown length recipe {lengths!r}")
+    else:
+        lens = torch.tensor([int(x) for x in lengths], dtype=torch.int32)
+        if lens.numel() != B:
+            raise ValueError("one length per sequence expected")
+    out["seqlens"] = lens
+    if tail_nan:
+        for b in range(B):
+            n = max(0, min(int(lens[b]), N_kv))
+            out["k"][b, n:] = float("nan")
+            out["v"][b, n:] = float("nan")
+    return out
+
+
+def make_decode_workload_inputs(w: DecodeWorkload) -> dict[str, torch.Tensor]:
+    return make_decode_inputs(w.B, w.H, w.H_kv, w.N_q, w.N_kv, w.d, w.seed, lengths=w.lengths)
+
+
 def peaked_positions(N: int, gen: torch.Generator) -> torch.Tensor:
     """floor(N/100) distinct sequence positions, drawn by a seeded permutation."""
     return torch.randperm(N, generator=gen)[: N // 100]

@@ -17,4 +17,5 @@ from .oracle import (  # noqa: F401
     dense_fwd,
     dense_bwd,
     online_fwd,
+    decode_rows,
 )

@@ -20,6 +20,9 @@ Three independent routes to the same numbers, all fp64, all on one head
   ("Flash Attention Explained", "Compute softmax incrementally"; holysheep.ai
   review, "the online softmax algorithm combined with tiling").  It exists to
   pin the claim that the streaming result equals the two-pass result.
+* ``decode_rows``: decoding -- N_q new queries per sequence, placed after a
+  cached prefix of per-sequence length, against a key/value cache; each
+  (sequence, head) is ``fwd_rows`` evaluated at the queries' positions.
 
 Causal: key j visible to query i iff j <= i.  LSE is the natural-log
 log-sum-exp of the scaled, visible scores.
@@ -28,7 +31,12 @@ Parity status: pinned (see ``tests/test_oracle_pins.py``): library softmax /
 logsumexp (scipy) on brute-force tiny inputs, logistic closed form at N=2,
 N=1 closed form, identical-score and dominant-score cases, rows of P summing
 to one, central finite differences of L = sum(O * dO) for the gradients,
-sum_j dK_j = 0, and online == two-pass.
+sum_j dK_j = 0, and online == two-pass.  ``decode_rows`` is pinned by scipy
+brute force over positions, head groups and cache lengths, by the NaN-filled
+cache tail changing nothing, by grouped == expanded heads, by the empty-row
+cases, and by equality with the whole-sequence rows of ``dense_fwd``
+(``tests/test_oracle_decode_pins.py``, which also plants five mistakes in a
+numpy copy and checks that each is caught).
 """
 from __future__ import annotations
 
@@ -231,3 +239,56 @@ def online_fwd(q, k, v, scale: float, causal: bool, tile_widths, window: int = -
         m = m_new
         start += w
     return acc / l[:, None], m + np.log(l)
+
+
+def decode_rows(q, k, v, seqlens, scale: float, causal: bool, window: int = -1, heads=None):
+    """Decoding: the outputs of N_q new queries per sequence against a key/value cache.
+
+    ``q``: [B, N_q, H, d]; ``k``, ``v``: [B, N_kv, H_kv, d], the cache, of which only the
+    first ``seqlens[b]`` positions of sequence b are real (``None``: all N_kv).  Query head
+    h reads key/value head h // (H // H_kv) ("Flash Attention Explained", institutepm.com,
+    "Grouped Query Attention").  With causal masking query i of sequence b stands at
+    position len_b - N_q + i, right after the cached prefix it extends, and sees the keys
+    at or before it (and, with a window, no more than ``window`` positions back); without
+    it every cached key is visible.  This is the generation phase the pages set against
+    prompt processing ("What Is Flash Attention?", bestllmfor.com, table "What you
+    actually gain on a local machine").
+
+    Each (b, h) is the plain definition of ``fwd_rows`` on one head: the queries are placed
+    at their positions in an otherwise empty query block of the sequence's length and only
+    those rows are evaluated.  A query that sees no key (empty cache, or a position before
+    the start) gets O = 0 and LSE = -inf.  ``heads`` restricts the work to a list of (b, h)
+    pairs; other outputs stay NaN.
+
+    Returns O (fp64 [B, N_q, H, d]) and LSE (fp64 [B, H, N_q]).
+    """
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    B, n_q, H, d = q.shape
+    n_kv, h_kv = k.shape[1], k.shape[2]
+    if k.shape != (B, n_kv, h_kv, d) or v.shape != k.shape or H % h_kv:
+        raise ValueError(f"bad decode shapes {q.shape}, {k.shape}, {v.shape}")
+    if window >= 0 and not causal:
+        raise ValueError("a window needs causal attention")
+    lens = np.full(B, n_kv, np.int64) if seqlens is None else np.clip(np.asarray(seqlens, np.int64), 0, n_kv)
+    group = H // h_kv
+    o = np.full((B, n_q, H, d), np.nan)
+    lse = np.full((B, H, n_q), np.nan)
+    todo = [(b, h) for b in range(B) for h in range(H)] if heads is None else [tuple(x) for x in heads]
+    for b, h in todo:
+        n = int(lens[b])
+        kh, vh = k[b, :n, h // group], v[b, :n, h // group]
+        o[b, :, h] = 0.0
+        lse[b, h] = -np.inf
+        if n == 0:
+            continue
+        for i in range(n_q):
+            pos = n - n_q + i if causal else 0
+            if pos < 0:
+                continue
+            qh = np.zeros((n, d))
+            qh[pos] = q[b, i, h]
+            oi, li = fwd_rows(qh, kh, vh, scale, causal, [pos], window)
+            o[b, i, h], lse[b, h, i] = oi[0], li[0]
+    return o, lse

@@ -275,3 +275,78 @@ def check_window_finite_differences(impl, seed=24, h=1e-6):
 
 ALL_WINDOW_CHECKS = [check_window_library_softmax, check_window_zero_closed_form,
                      check_window_past_blind, check_window_finite_differences]
+
+
+# ---------------------------------------------------------------- decoding against a cache
+# Each check takes ``decode(q, k, v, seqlens, scale, causal, window=-1) -> (O, LSE)`` with
+# q [B, N_q, H, d], k/v [B, N_kv, H_kv, d], O [B, N_q, H, d] and LSE [B, H, N_q].
+
+def _decode_case(rng, B, n_q, H, h_kv, n_kv, d):
+    return (_bf16_grid(rng.standard_normal((B, n_q, H, d))),
+            _bf16_grid(rng.standard_normal((B, n_kv, h_kv, d))),
+            _bf16_grid(rng.standard_normal((B, n_kv, h_kv, d))))
+
+
+def check_decode_library_softmax(decode, seed=41):
+    """Brute force against scipy: the queries are the last N_q positions of each cached
+    sequence, query head h reads key/value head h // (H / H_kv), and only the first
+    seqlens[b] cache positions exist."""
+    rng = _rng(seed)
+    B, n_q, H, h_kv, n_kv, d = 3, 3, 4, 2, 13, 5
+    lens = [13, 6, 3]
+    q, k, v = _decode_case(rng, B, n_q, H, h_kv, n_kv, d)
+    for causal, window in ((True, -1), (False, -1), (True, 0), (True, 2), (True, 4)):
+        o, lse = decode(q, k, v, lens, 0.6, causal, window)
+        for b in range(B):
+            n = lens[b]
+            for h in range(H):
+                kv = h // (H // h_kv)
+                for i in range(n_q):
+                    pos = n - n_q + i
+                    keys = [j for j in range(n)
+                            if not causal or (j <= pos and (window < 0 or j >= pos - window))]
+                    s = np.array([0.6 * sum(q[b, i, h, x] * k[b, j, kv, x] for x in range(d)) for j in keys])
+                    p = softmax(s)
+                    o_ref = sum(p[t] * v[b, j, kv] for t, j in enumerate(keys))
+                    np.testing.assert_allclose(o[b, i, h], o_ref, rtol=0, atol=1e-12)
+                    np.testing.assert_allclose(lse[b, h, i], logsumexp(s), rtol=1e-13, atol=1e-13)
+
+
+def check_decode_cache_tail_ignored(decode, seed=42):
+    """Cache positions past a sequence's length do not exist: NaN there changes nothing."""
+    rng = _rng(seed)
+    q, k, v = _decode_case(rng, 2, 2, 2, 1, 9, 4)
+    lens = [5, 9]
+    o1, l1 = decode(q, k, v, lens, 0.5, True)
+    k2, v2 = k.copy(), v.copy()
+    k2[0, 5:] = np.nan
+    v2[0, 5:] = np.nan
+    o2, l2 = decode(q, k2, v2, lens, 0.5, True)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def check_decode_grouped_equals_expanded(decode, seed=43):
+    """Grouped key/value heads give what the same cache repeated per query head gives."""
+    rng = _rng(seed)
+    q, k, v = _decode_case(rng, 2, 2, 6, 2, 7, 4)
+    og, lg = decode(q, k, v, [7, 4], 0.4, True)
+    oe, le = decode(q, np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2), [7, 4], 0.4, True)
+    np.testing.assert_allclose(og, oe, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lg, le, rtol=0, atol=1e-14)
+
+
+def check_decode_empty_rows(decode, seed=44):
+    """An empty cache, or a query placed before the start of its sequence, sees no key:
+    O = 0 and LSE = -inf; the other rows are unaffected."""
+    rng = _rng(seed)
+    q, k, v = _decode_case(rng, 2, 3, 1, 1, 6, 3)
+    o, lse = decode(q, k, v, [0, 2], 0.5, True)
+    assert np.all(o[0] == 0) and np.all(lse[0] == -np.inf)
+    assert np.all(o[1, 0] == 0) and lse[1, 0, 0] == -np.inf
+    # the second query of sequence 1 stands at position 0 and sees only key 0
+    np.testing.assert_allclose(o[1, 1, 0], v[1, 0, 0], rtol=0, atol=1e-15)
+    assert np.isfinite(lse[1, 0, 1]) and np.isfinite(lse[1, 0, 2])
+
+
+ALL_DECODE_CHECKS = [check_decode_library_softmax, check_decode_cache_tail_ignored,
+                     check_decode_grouped_equals_expanded, check_decode_empty_rows]

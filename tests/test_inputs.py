@@ -44,3 +44,21 @@ def test_workloads_table():
     w = WORKLOADS["causal_fwdbwd_b2_h16_n8192_d128"]
     assert (w.B, w.H, w.N, w.d, w.causal, w.backward) == (2, 16, 8192, 128, True, True)
     assert abs(w.scale - 128 ** -0.5) < 1e-15
+
+
+def test_decode_inputs_recipe():
+    from exact_io_aware_93_b200.inputs import DECODE_WORKLOADS, make_decode_inputs
+    a = make_decode_inputs(3, 4, 2, 2, 300, 64, 5, lengths="mixed")
+    b = make_decode_inputs(3, 4, 2, 2, 300, 64, 5, lengths="mixed")
+    assert a["q"].shape == (3, 2, 4, 64) and a["k"].shape == (3, 300, 2, 64)
+    for n in ("q", "k", "v", "seqlens"):
+        assert torch.equal(a[n], b[n])
+    assert a["seqlens"].dtype == torch.int32
+    assert torch.all((a["seqlens"] >= 150) & (a["seqlens"] <= 300))
+    full = make_decode_inputs(3, 4, 2, 2, 300, 64, 5, lengths="full")
+    assert torch.equal(full["q"], a["q"]) and torch.all(full["seqlens"] == 300)
+    t = make_decode_inputs(2, 2, 1, 1, 10, 8, 6, lengths=[4, 10], tail_nan=True)
+    assert torch.isnan(t["k"][0, 4:]).all() and not torch.isnan(t["k"][0, :4]).any()
+    assert not torch.isnan(t["v"][1]).any()
+    w = next(iter(DECODE_WORKLOADS.values()))
+    assert w.N_kv % 128 == 0 and w.H % w.H_kv == 0
