@@ -35,11 +35,14 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from exact_io_aware_93_b200.accounting import bwd_flops_window, fwd_bytes, fwd_flops_window  # noqa: E402
-from exact_io_aware_93_b200.inputs import EXTRA_WORKLOADS, WORKLOADS, make_inputs  # noqa: E402
+from exact_io_aware_93_b200.accounting import (bwd_flops_window, decode_bytes, decode_flops, fwd_bytes,  # noqa: E402
+                                                fwd_flops_window)
+from exact_io_aware_93_b200.inputs import (DECODE_WORKLOADS, EXTRA_WORKLOADS, WORKLOADS,  # noqa: E402
+                                           make_decode_workload_inputs, make_inputs)
 from exact_io_aware_93_b200.replicas import max_over_ranks, whole_job_tflops, world as _world  # noqa: E402
 
 METRIC = "attention fwd/bwd TFLOPS and % of B200 dense-bf16 peak, causal N=2K–128K"
+DECODE_METRIC = "attention decode: key/value cache bytes streamed per second (GB/s) and % of B200 HBM bandwidth"
 DEFAULT_WORKLOAD = "causal_fwdbwd_b2_h16_n8192_d128"
 L2_BYTES = 126 * 1024 * 1024
 
@@ -408,17 +411,181 @@ def run_ours(args, w):
     return 0
 
 
+def _decode_sample_heads(w, count):
+    return [(b % w.B, (7 * b + 3) % w.H) for b in range(count)]
+
+
+def decode_cpu_sample(w, inp, pairs, threads):
+    """Time the fp64 oracle's decode on the given (b, h) pairs; returns (bytes, seconds) with
+    bytes counted like decode_bytes for those heads (each head's key/value rows once)."""
+    import oracle
+    oracle.oracle_threads(threads)
+    q, k, v = (inp[n].double().numpy() for n in ("q", "k", "v"))
+    lens = inp["seqlens"].numpy()
+    t0 = time.perf_counter()
+    oracle.decode_rows(q, k, v, lens, w.scale, w.causal, w.window, heads=pairs)
+    dt = time.perf_counter() - t0
+    nbytes = sum(decode_bytes([lens[b]], 1, 1, 1, w.N_q, w.d, w.causal, w.window) for b, _ in pairs)
+    return nbytes, dt
+
+
+def run_decode(args, w):
+    """Decoding workload: one step = one fa_decode call (split-KV kernel + merge kernel)."""
+    world, rank, local = _dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        threads = len(os.sched_getaffinity(0))
+        inp = make_decode_workload_inputs(w)
+        per_step = REFERENCE_BUDGET_S / (args.warmup + args.steps)
+        nb, dt = decode_cpu_sample(w, inp, _decode_sample_heads(w, 1), threads)
+        heads = max(1, min(w.B * w.H, int(per_step / max(dt, 1e-6))))
+        pairs = _decode_sample_heads(w, heads)
+        times, nbytes = [], 0
+        for i in range(args.warmup + args.steps):
+            nbytes, dt = decode_cpu_sample(w, inp, pairs, threads)
+            if i >= args.warmup:
+                times.append(dt)
+        value = nbytes * len(times) / sum(times) / 1e9
+        line = {
+            "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N_q": w.N_q, "N_kv": w.N_kv,
+                       "d": w.d, "causal": w.causal, "window": w.window},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": f"oracle decode of {len(pairs)} (sequence, head) pairs of {w.name} per step"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from exact_io_aware_93_b200 import api
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = make_decode_workload_inputs(w)
+    t = {n: inp[n].to(dev) for n in ("q", "k", "v", "seqlens")}
+    t["o"] = torch.empty_like(t["q"])
+    t["lse"] = torch.empty((w.B, w.H, w.N_q), dtype=torch.float32, device=dev)
+    t["ws"] = torch.empty(api.decode_workspace_size(t["q"], t["k"], w.causal, _win(w)), dtype=torch.uint8,
+                          device=dev)
+    lens = inp["seqlens"].tolist()
+    step_bytes = decode_bytes(lens, w.B, w.H, w.H_kv, w.N_q, w.d, w.causal, w.window)
+    step_flops = decode_flops(lens, w.H, w.N_q, w.d, w.causal, w.window)
+    cache_bytes = 2 * t["k"].numel() * t["k"].element_size()
+
+    def step():
+        api.decode(t["q"], t["k"], t["v"], t["seqlens"], causal=w.causal, out=t["o"], lse=t["lse"],
+                   workspace=t["ws"], window=_win(w))
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if api.get_status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_begin = time.time()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    t_end = time.time()
+    if world > 1:
+        dist.barrier()
+    clocks.mark(t_begin, t_end)
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    status = api.get_status()
+
+    # end to end through the public API: the new queries and lengths come from pinned host
+    # memory and O, LSE go back every step; the cache stays resident on the device
+    host_in = {n: inp[n].pin_memory() for n in ("q", "seqlens")}
+    host_out = {n: torch.empty(t[n].shape, dtype=t[n].dtype).pin_memory() for n in ("o", "lse")}
+    h2d = sum(x.numel() * x.element_size() for x in host_in.values())
+    d2h = sum(x.numel() * x.element_size() for x in host_out.values())
+
+    def e2e_step():
+        for n, x in host_in.items():
+            t[n].copy_(x, non_blocking=True)
+        step()
+        for n, x in host_out.items():
+            x.copy_(t[n], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(1, min(args.steps, 50))
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    if world > 1:
+        ms, e2e_ms = max_over_ranks([ms, e2e_ms], dev)
+    _, _, hbm, peak_kind = _peaks()
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    value = world * gbs
+    line = {
+        "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N_q": w.N_q, "N_kv": w.N_kv,
+                   "d": w.d, "causal": w.causal, "window": w.window, "seqlens": lens,
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"not flushed: key/value cache {cache_bytes / 1e6:.0f} MB > L2 {L2_BYTES / 1e6:.0f} MB",
+                   "step": "fa_decode (split-KV kernel + merge kernel)"},
+        "tokens_per_s": world * w.B * w.N_q / (ms * 1e-3),
+        "tflops": world * step_flops / (ms * 1e-3) / 1e12,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "traffic": measured_traffic("fa_decode", w.name), "kernel": "fa_decode (kernel + merge)",
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth", "alg_bytes_per_launch": step_bytes},
+        "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
+        "gpu_launches": args.steps * 2,
+        "clocks": clk,
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = len(os.sched_getaffinity(0))
+        pairs = _decode_sample_heads(w, 16)
+        nb, dt = decode_cpu_sample(w, inp, pairs, threads)
+        line["cpu_baseline"] = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                "sample": f"oracle decode of {len(pairs)} (sequence, head) pairs of {w.name}, "
+                                          f"fp64, {dt:.1f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS) + sorted(EXTRA_WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(WORKLOADS) + sorted(EXTRA_WORKLOADS) + sorted(DECODE_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.workload in DECODE_WORKLOADS:
+        return run_decode(args, DECODE_WORKLOADS[args.workload])
     w = {**WORKLOADS, **EXTRA_WORKLOADS}[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)

@@ -52,3 +52,33 @@ def fwd_flops_window(B: int, H: int, N: int, d: int, causal: bool, window: int =
 
 def bwd_flops_window(B: int, H: int, N: int, d: int, causal: bool, window: int = -1) -> float:
     return 2.5 * fwd_flops_window(B, H, N, d, causal, window)
+
+
+def decode_cache_keys(length: int, N_q: int, causal: bool, window: int = -1) -> int:
+    """Cache positions of one sequence that some new query can see: all `length` of them,
+    or with a causal window the last N_q + window (fewer when the cache is shorter)."""
+    n = max(0, int(length))
+    if causal and window >= 0:
+        return min(n, N_q + window)
+    return n
+
+
+def decode_bytes(seqlens, B: int, H: int, H_kv: int, N_q: int, d: int, causal: bool, window: int = -1) -> int:
+    """Algorithmic bytes of one decode call: the visible K and V cache rows of every
+    key/value head read once (bf16), Q read and O written (bf16), LSE written (fp32) and
+    the lengths read (int32)."""
+    keys = sum(decode_cache_keys(n, N_q, causal, window) for n in seqlens)
+    return 2 * 2 * keys * H_kv * d + 2 * 2 * B * N_q * H * d + 4 * B * H * N_q + 4 * B
+
+
+def decode_flops(seqlens, H: int, N_q: int, d: int, causal: bool, window: int = -1) -> float:
+    """4*d flops per visible (query, key) pair and query head."""
+    pairs = 0
+    for n in seqlens:
+        n = max(0, int(n))
+        for i in range(N_q):
+            pos = n - N_q + i if causal else n - 1
+            if pos < 0:
+                continue
+            pairs += (min(pos, window) + 1) if (causal and window >= 0) else (pos + 1 if causal else n)
+    return 4.0 * d * H * pairs

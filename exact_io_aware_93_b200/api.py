@@ -33,6 +33,13 @@ class FaProblem(ctypes.Structure):
                 ("window", ctypes.c_int)]
 
 
+class FaDecodeProblem(ctypes.Structure):
+    """The ``fa_decode_problem`` descriptor of include/fa.h."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int), ("N_q", ctypes.c_int),
+                ("N_kv", ctypes.c_int), ("d", ctypes.c_int), ("scale", ctypes.c_float),
+                ("causal", ctypes.c_int), ("window", ctypes.c_int)]
+
+
 class FAError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = int(status)
@@ -76,6 +83,10 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
                          i, i, i, i, f, i, vp]
     L.fa_bwd.restype = i
+    L.fa_decode_workspace_size.argtypes = [ctypes.POINTER(FaDecodeProblem)]
+    L.fa_decode_workspace_size.restype = ctypes.c_size_t
+    L.fa_decode.argtypes = [ctypes.POINTER(FaDecodeProblem), vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    L.fa_decode.restype = i
     _lib = L
     return L
 
@@ -170,6 +181,58 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, do: 
     if st != 0:
         raise FAError(st, "fa_bwd_ex")
     return dq, dk, dv
+
+
+def decode_problem(q: torch.Tensor, k_cache: torch.Tensor, causal: bool, scale: float | None,
+                   window: int | None) -> FaDecodeProblem:
+    B, n_q, H, d = q.shape
+    return FaDecodeProblem(B, H, k_cache.shape[2], n_q, k_cache.shape[1], d,
+                           1.0 / math.sqrt(d) if scale is None else float(scale), int(bool(causal)),
+                           -1 if window is None else int(window))
+
+
+def decode_workspace_size(q: torch.Tensor, k_cache: torch.Tensor, causal: bool = True,
+                          window: int | None = None) -> int:
+    """Bytes of device workspace ``fa_decode`` needs for these shapes on the current device."""
+    return int(lib().fa_decode_workspace_size(ctypes.byref(decode_problem(q, k_cache, causal, None, window))))
+
+
+def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+           seqlens: torch.Tensor | None = None, causal: bool = True, scale: float | None = None,
+           out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+           workspace: torch.Tensor | None = None, window: int | None = None):
+    """(O [B, N_q, H, d] bf16, LSE [B, H, N_q] fp32) of N_q new queries per sequence against a
+    key/value cache ``[B, N_kv, H_kv, d]`` via ``fa_decode``.
+
+    ``seqlens`` (int32 [B] on the device, or None for full caches) gives each sequence's cached
+    length; with ``causal`` the queries are the last N_q positions of each sequence: query i
+    of sequence b stands at position seqlens[b] - N_q + i."""
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if not isinstance(t, torch.Tensor) or t.dim() != 4 or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a 4-d bfloat16 tensor")
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor (no CPU path)")
+    B, n_q, H, d = q.shape
+    if k_cache.shape != v_cache.shape or k_cache.shape[0] != B or k_cache.shape[3] != d:
+        raise ValueError(f"cache shapes {tuple(k_cache.shape)}, {tuple(v_cache.shape)} do not fit q {tuple(q.shape)}")
+    if H % k_cache.shape[2] != 0:
+        raise ValueError("key/value heads must divide the query heads")
+    if seqlens is not None and (seqlens.dtype != torch.int32 or seqlens.shape != (B,) or not seqlens.is_cuda
+                                or not seqlens.is_contiguous()):
+        raise ValueError("seqlens must be a contiguous int32 [B] CUDA tensor")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, n_q), dtype=torch.float32, device=q.device) if lse is None else lse
+    p = decode_problem(q, k_cache, causal, scale, window)
+    need = int(lib().fa_decode_workspace_size(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib().fa_decode(ctypes.byref(p), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                         None if seqlens is None else seqlens.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                         workspace.data_ptr(), ws_bytes, _stream_ptr(q))
+    if st != 0:
+        raise FAError(st, "fa_decode")
+    return out, lse
 
 
 def get_status(device: torch.device | None = None) -> int:

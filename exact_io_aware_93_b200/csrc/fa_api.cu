@@ -9,6 +9,7 @@
 
 #include "../../include/fa.h"
 #include "fa_bwd_kernel.cuh"
+#include "fa_decode_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 #include "tma_host.h"
 
@@ -26,6 +27,7 @@ struct DeviceInfo {
   int* status = nullptr;
   bool fwd_attr[2][2] = {{false, false}, {false, false}};  // [d==128][causal]
   bool bwd_attr[2][2] = {{false, false}, {false, false}};
+  bool dec_attr[2] = {false, false};  // [d==128]
 };
 DeviceInfo g_dev[kMaxDevices];
 
@@ -162,6 +164,82 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   return FA_OK;
 }
 
+// ---------------------------------------------------------------- decoding
+fa_status check_decode(const fa_decode_problem& p) {
+  if (p.B < 1 || p.H < 1 || p.H_kv < 1 || p.N_q < 1 || p.N_kv < 1) return FA_ERR_INVALID_ARG;
+  if (p.H_kv > p.H || p.H % p.H_kv != 0) return FA_ERR_INVALID_ARG;
+  if (!(p.scale > 0.0f) || !isfinite(p.scale)) return FA_ERR_INVALID_ARG;
+  if (p.causal != 0 && p.causal != 1) return FA_ERR_INVALID_ARG;
+  if (p.window < -1 || (p.window >= 0 && p.causal != 1)) return FA_ERR_INVALID_ARG;
+  if (p.d != 64 && p.d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p.H / p.H_kv) * p.N_q > fa::kDecMaxRows) return FA_ERR_UNSUPPORTED;
+  // tile counts, tile starts and element offsets stay in range
+  const long long tiles = static_cast<long long>(p.B) * p.H_kv * ((static_cast<long long>(p.N_kv) + 127) / 128);
+  if (tiles > (1ll << 30)) return FA_ERR_INVALID_ARG;
+  if (static_cast<long double>(p.B) * p.N_kv * p.H_kv * p.d > static_cast<long double>(INT64_MAX / 4))
+    return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct DecLayout {
+  size_t meta, part_lse, part_o, total;
+};
+
+// Workspace regions: schedule (total, tiles per CTA, per-sequence prefix), then the
+// partial log-sum-exps [S, M, 2] and partial outputs [S, M, d] of S = grid + B*H_kv - 1
+// slots (slot = CTA index + pair index is unique along the flattened tile list).
+DecLayout dec_layout(const fa_decode_problem& p, int grid) {
+  const size_t M = static_cast<size_t>(p.H / p.H_kv) * p.N_q;
+  const size_t slots = static_cast<size_t>(grid) + static_cast<size_t>(p.B) * p.H_kv - 1;
+  DecLayout L;
+  L.meta = 0;
+  L.part_lse = round256((2 + static_cast<size_t>(p.B)) * 4);
+  L.part_o = L.part_lse + round256(slots * M * 2 * 4);
+  L.total = L.part_o + slots * M * static_cast<size_t>(p.d) * 4;
+  return L;
+}
+
+template <int D>
+fa_status launch_decode(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const fa_decode_problem& p, const int* seqlens, void* o, float* lse, void* ws,
+                        cudaStream_t stream) {
+  auto kern = fa::fa_decode_kernel<D>;
+  const int smem = static_cast<int>(sizeof(fa::DecSmem<D>)) + 1024;
+  bool& attr = di.dec_attr[D == 128];
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    attr = true;
+  }
+  const int grid = di.sm_count;
+  const DecLayout L = dec_layout(p, grid);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  fa::DecArgs a;
+  a.seqlens = seqlens;
+  a.out = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.meta = reinterpret_cast<int*>(w + L.meta);
+  a.part_lse = reinterpret_cast<float*>(w + L.part_lse);
+  a.part_o = reinterpret_cast<float*>(w + L.part_o);
+  a.B = p.B;
+  a.H = p.H;
+  a.H_kv = p.H_kv;
+  a.N_q = p.N_q;
+  a.N_kv = p.N_kv;
+  a.window = p.window;
+  a.causal = p.causal;
+  a.scale_log2 = p.scale * 1.4426950408889634f;
+  kern<<<grid, fa::kDecThreads, smem, stream>>>(mq, mk, mv, a, di.status);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  fa::fa_decode_merge_kernel<D><<<p.B * p.H_kv, 128, 0, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
 // ---------------------------------------------------------------- wait-timeout self-test
 // One warp waits on an mbarrier that nothing will ever arrive on, with the given bound,
 // through the same bounded-wait path the attention kernels use.  The wait runs out, the
@@ -220,7 +298,7 @@ fa_status noalloc_scratch(void** out) {
 
 extern "C" {
 
-int fa_abi_version(void) { return 2; }
+int fa_abi_version(void) { return 3; }
 
 const char* fa_status_string(int s) {
   switch (s) {
@@ -332,6 +410,39 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   const fa_status ss = noalloc_scratch(&scratch);
   if (ss != FA_OK) return ss;
   return fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, scratch, kNoAllocScratchBytes, B, H, N, d, scale, causal, stream);
+}
+
+size_t fa_decode_workspace_size(const fa_decode_problem* problem) {
+  if (!problem || check_decode(*problem) != FA_OK) return 0;
+  DeviceInfo* di = nullptr;
+  if (current_device(&di) != FA_OK) return 0;
+  return dec_layout(*problem, di->sm_count).total;
+}
+
+fa_status fa_decode(const fa_decode_problem* problem, const void* q, const void* k_cache, const void* v_cache,
+                    const int* seqlens, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  if (!problem || !q || !k_cache || !v_cache || !o || !lse) return FA_ERR_INVALID_ARG;
+  const fa_decode_problem p = *problem;
+  fa_status st = check_decode(p);
+  if (st != FA_OK) return st;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(seqlens, 4))
+    return FA_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  st = current_device(&di);
+  if (st != FA_OK) return st;
+  if (workspace == nullptr || workspace_bytes < dec_layout(p, di->sm_count).total) return FA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return FA_ERR_ALIGNMENT;
+  const int G = p.H / p.H_kv;
+  CUtensorMap mq, mk, mv;
+  if (!fa::make_decode_q_map(&mq, q, p.B, p.N_q, p.H, p.d, G) ||
+      !fa::make_bshd_map(&mk, k_cache, p.B, p.N_kv, p.H_kv, p.d, 128) ||
+      !fa::make_bshd_map(&mv, v_cache, p.B, p.N_kv, p.H_kv, p.d, 128))
+    return FA_ERR_LAUNCH;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p.d == 128) return launch_decode<128>(*di, mq, mk, mv, p, seqlens, o, lse, workspace, s);
+  return launch_decode<64>(*di, mq, mk, mv, p, seqlens, o, lse, workspace, s);
 }
 
 fa_status fa_selftest_wait_timeout(unsigned int timeout_us, void* stream) {

@@ -41,6 +41,23 @@ inline bool make_bshd_map(CUtensorMap* map, const void* base, int B, int N, int 
   return r == CUDA_SUCCESS;
 }
 
+// Decoding queries [B, N_q, H, d]: one box holds the G consecutive heads starting at a
+// given head for all N_q positions of one sequence, 64 columns wide.  In shared memory it
+// lands as rows r = i * G + g of 128 bytes (128-byte swizzle), the row order of a
+// 128-row MMA tile.
+inline bool make_decode_q_map(CUtensorMap* map, const void* base, int B, int N_q, int H, int d, int G) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N_q, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)N_q * H * d * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)N_q, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // A row-major [rows, cols] bf16 matrix as a 2-D map with boxes of box_rows x 64 columns (128-byte swizzle).
 inline bool make_2d_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
   EncodeTiledFn enc = encode_tiled_fn();

@@ -56,7 +56,7 @@ typedef enum {
   FA_ERR_WORKSPACE = 7    /* workspace pointer NULL or smaller than the required size */
 } fa_status;
 
-/* Library ABI version (this header: 2). */
+/* Library ABI version (this header: 3). */
 int fa_abi_version(void);
 
 /*
@@ -165,6 +165,72 @@ fa_status fa_bwd_ex(const fa_problem* problem, const void* q, const void* k, con
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
                          int causal, void* stream);
+
+/*
+ * ---------------------------------------------------------------- decoding
+ * Attention of a few NEW queries per sequence against a key/value cache: the generation
+ * phase, as opposed to prompt processing ("What Is Flash Attention?", bestllmfor.com,
+ * table "What you actually gain on a local machine").  The result is the same exact
+ * softmax(scale * q K^T) V over each query's visible cached keys; the cache is split
+ * over all SMs and the pieces are combined by their log-sum-exps.
+ *
+ *   B        : sequences
+ *   H, H_kv  : query heads and key/value heads (H % H_kv == 0; query head h reads
+ *              key/value head h / (H / H_kv))
+ *   N_q      : new queries per sequence, 1 for plain decoding (more for, e.g., verifying
+ *              several drafted tokens at once)
+ *   N_kv     : cache capacity: positions per sequence in k_cache / v_cache
+ *   d        : 64 or 128
+ *   scale    : softmax scale (> 0, finite)
+ *   causal   : 1: query i of sequence b stands at position len_b - N_q + i, right after
+ *              the cached prefix it extends, and sees the cached keys at or before that
+ *              position; 0: every query sees all len_b cached keys
+ *   window   : -1, or >= 0 with causal = 1: a query at position t sees keys t - window .. t
+ * Constraint: (H / H_kv) * N_q <= 128 (the rows one key/value head contributes to a
+ * 128-row tile); larger groups return FA_ERR_UNSUPPORTED.
+ */
+typedef struct fa_decode_problem {
+  int B;
+  int H;
+  int H_kv;
+  int N_q;
+  int N_kv;
+  int d;
+  float scale;
+  int causal;
+  int window;
+} fa_decode_problem;
+
+/*
+ * Bytes of device workspace fa_decode needs on the CURRENT device (the split over its SMs
+ * sets the number of partial results): 256-byte-aligned regions for the schedule
+ * (4 * (2 + B) bytes), the partial log-sum-exps (8 * S * M) and the partial outputs
+ * (4 * S * M * d), with S = SMs + B * H_kv - 1 and M = (H / H_kv) * N_q.
+ * Returns 0 for an invalid or unsupported problem or without an sm_100 device.
+ */
+size_t fa_decode_workspace_size(const fa_decode_problem* problem);
+
+/*
+ * Decoding forward.
+ *   q        : in,  bf16 [B, N_q, H, d]
+ *   k_cache  : in,  bf16 [B, N_kv, H_kv, d]; only the first len_b positions of sequence b
+ *              are read as keys: the rest may hold anything (stale values, NaN)
+ *   v_cache  : in,  bf16 [B, N_kv, H_kv, d], same rule
+ *   seqlens  : in,  DEVICE int32 [B]: len_b, the cached length of each sequence (values
+ *              are clamped to [0, N_kv]), or NULL: every sequence is N_kv long.  Read by
+ *              the kernels, so a captured CUDA graph can be replayed as lengths grow.
+ *   o        : out, bf16 [B, N_q, H, d]
+ *   lse      : out, fp32 [B, H, N_q], natural-log log-sum-exp of each query's visible scores
+ *   workspace: device scratch of at least fa_decode_workspace_size() bytes, 256-byte
+ *              aligned; contents on entry do not matter
+ * A query that sees no key (len_b = 0, or a position before the start of the cache) gets
+ * O = 0 and LSE = -inf.  Deterministic for fixed inputs and device.  Errors: as fa_fwd,
+ * FA_ERR_INVALID_ARG for a bad problem (a window without causal masking included),
+ * FA_ERR_UNSUPPORTED beyond the constraint above, FA_ERR_ALIGNMENT, FA_ERR_WORKSPACE.
+ */
+fa_status fa_decode(const fa_decode_problem* problem, const void* q, const void* k_cache, const void* v_cache,
+                    const int* seqlens, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                    void* stream);
 
 /*
  * Failure-detection self-test: launches one warp that waits on a barrier nothing will

@@ -130,3 +130,31 @@ def grad_errors_gqa(inputs, grads_gpu, scale, causal, window=-1):
                 num[name] = max(num[name], float(np.abs(got - ref).max()))
                 den[name] = max(den[name], float(np.abs(ref).max()))
     return {n: num[n] / max(den[n], GRAD_ABS_FLOOR) for n in num}
+
+
+def decode_errors(inputs, o_gpu, lse_gpu, scale, causal, window=-1, heads=None):
+    """(O error, LSE error) of a decode call against ``oracle.decode_rows`` over the given
+    (b, h) pairs (default: all).  O: excess over half a bf16 ulp, as for the grouped rows;
+    LSE: relative as everywhere, and -inf exactly where the oracle has -inf (no key seen)."""
+    q = inputs["q"].double().numpy()
+    k = inputs["k"].double().numpy()
+    v = inputs["v"].double().numpy()
+    o_ref, lse_ref = oracle.decode_rows(q, k, v, inputs["seqlens"].numpy(), scale, causal, window, heads=heads)
+    B, n_q, H, _ = q.shape
+    pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    o_g = o_gpu.cpu().double().numpy()
+    l_g = lse_gpu.cpu().double().numpy()
+    worst_o, worst_l = 0.0, 0.0
+    for b, h in pairs:
+        og, orf = o_g[b, :, h], o_ref[b, :, h]
+        lg, lrf = l_g[b, h], lse_ref[b, h]
+        if not np.all(np.isfinite(og)):
+            return float("inf"), float("inf")
+        empty = np.isneginf(lrf)
+        if not np.array_equal(np.isneginf(lg), empty):
+            return float("inf"), float("inf")
+        worst_o = max(worst_o, float((np.abs(og - orf) - bf16_half_ulp(orf)).max()))
+        if (~empty).any():
+            worst_l = max(worst_l, float((np.abs(lg[~empty] - lrf[~empty]) /
+                                          np.maximum(1.0, np.abs(lrf[~empty]))).max()))
+    return worst_o, worst_l

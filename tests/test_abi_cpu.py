@@ -46,7 +46,7 @@ def test_status_strings(lib):
     assert lib.fa_status_string(0) == b"FA_OK"
     assert lib.fa_status_string(6) == b"FA_ERR_TIMEOUT"
     assert lib.fa_status_string(99) == b"FA_ERR_UNKNOWN"
-    assert lib.fa_abi_version() == 2
+    assert lib.fa_abi_version() == 3
 
 
 def _fwd(lib, q=0x10000, k=0x10000, v=0x10000, o=0x10000, lse=0x10000, B=1, H=1, N=16, d=64,
@@ -137,3 +137,38 @@ def test_ex_validation_codes(lib):
     assert fwd(d=96) == 2
     p = FaProblem(2, 4, 1, 100, 128, 0.1, 1, 16)
     assert lib.fa_bwd_workspace_size_ex(ctypes.byref(p)) == 4 * 2 * 4 * (100 * 128 + 2 * 128)
+
+
+def test_decode_validation_codes(lib):
+    """fa_decode checks its problem and pointers on the host, before any device work."""
+    from exact_io_aware_93_b200.api import FaDecodeProblem
+    vp = ctypes.c_void_p
+    lib.fa_decode.argtypes = [ctypes.POINTER(FaDecodeProblem), vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.fa_decode.restype = ctypes.c_int
+    lib.fa_decode_workspace_size.argtypes = [ctypes.POINTER(FaDecodeProblem)]
+    lib.fa_decode_workspace_size.restype = ctypes.c_size_t
+    P = 0x10000
+
+    def dec(seqlens=None, q=P, lse=P, **kw):
+        base = dict(B=2, H=8, H_kv=2, N_q=1, N_kv=1000, d=128, scale=0.1, causal=1, window=-1)
+        base.update(kw)
+        p = FaDecodeProblem(**base)
+        return lib.fa_decode(ctypes.byref(p), vp(q), vp(P), vp(P), None if seqlens is None else vp(seqlens),
+                             vp(P), vp(lse), vp(P), 1 << 30, None)
+    assert lib.fa_decode(None, vp(P), vp(P), vp(P), None, vp(P), vp(P), vp(P), 0, None) == 1
+    assert dec(q=0) == 1
+    assert dec(B=0) == 1 and dec(N_q=0) == 1 and dec(N_kv=0) == 1
+    assert dec(H_kv=3) == 1 and dec(H_kv=16) == 1
+    assert dec(scale=0.0) == 1 and dec(causal=2) == 1
+    assert dec(window=-2) == 1 and dec(window=4, causal=0) == 1
+    assert dec(d=96) == 2
+    assert dec(H=8, H_kv=1, N_q=17) == 2       # 8 heads x 17 positions > 128 rows
+    assert dec(H=8, H_kv=1, N_q=16) != 2
+    assert dec(q=P + 8) == 3
+    assert dec(lse=P + 2) == 3
+    assert dec(seqlens=P + 2) == 3
+    import torch
+    if not torch.cuda.is_available():
+        assert dec() == 4                       # valid problem, no sm_100 device here
+        p = FaDecodeProblem(2, 8, 2, 1, 1000, 128, 0.1, 1, -1)
+        assert lib.fa_decode_workspace_size(ctypes.byref(p)) == 0
