@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 from exact_io_aware_93_b200.accounting import (bwd_flops_window, decode_bytes, decode_flops, fwd_bytes,  # noqa: E402
                                                 fwd_flops_window)
 from exact_io_aware_93_b200.inputs import (DECODE_WORKLOADS, EXTRA_WORKLOADS, WORKLOADS,  # noqa: E402
-                                           make_decode_workload_inputs, make_inputs)
+                                           make_decode_workload_inputs, make_inputs, make_workload_inputs)
 from exact_io_aware_93_b200.replicas import max_over_ranks, whole_job_tflops, world as _world  # noqa: E402
 
 METRIC = "attention fwd/bwd TFLOPS and % of B200 dense-bf16 peak, causal N=2K–128K"
@@ -174,7 +174,11 @@ def _step_fn(api, t, w, with_bwd, events=None):
         if events is not None:
             events["fwd"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
             events["fwd"][-1][0].record()
-        api.fwd(t["q"], t["k"], t["v"], causal=w.causal, out=t["o"], lse=t["lse"], window=_win(w))
+        if w.dtype == "e4m3":
+            api.fwd_e4m3(t["q"], t["k"], t["v"], t["q_descale"], t["k_descale"], t["v_descale"],
+                         causal=w.causal, out=t["o"], lse=t["lse"], window=_win(w))
+        else:
+            api.fwd(t["q"], t["k"], t["v"], causal=w.causal, out=t["o"], lse=t["lse"], window=_win(w))
         if events is not None:
             events["fwd"][-1][1].record()
         if with_bwd:
@@ -284,16 +288,25 @@ def run_ours(args, w):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     from exact_io_aware_93_b200 import api
     dev = torch.device("cuda", torch.cuda.current_device())
-    with_bwd = with_bwd_available()
+    is8 = w.dtype == "e4m3"             # the e4m3 path is forward only
+    with_bwd = with_bwd_available() and not is8
 
-    inp = make_inputs(w.B, w.H, w.N, w.d, w.seed, with_do=True, peaked=w.peaked, H_kv=w.H_kv)
-    t = {n: inp[n].to(dev) for n in ("q", "k", "v", "do")}
-    t["o"] = torch.empty_like(t["q"])
+    if is8:
+        inp = make_workload_inputs(w)
+        names = ("q", "k", "v")
+    else:
+        inp = make_inputs(w.B, w.H, w.N, w.d, w.seed, with_do=True, peaked=w.peaked, H_kv=w.H_kv,
+                          dtype=w.torch_dtype)
+        names = ("q", "k", "v", "do")
+    t = {n: inp[n].to(dev) for n in names}
+    if is8:
+        t.update({n: inp[n] for n in ("q_descale", "k_descale", "v_descale")})
+    t["o"] = torch.empty(t["q"].shape, dtype=torch.bfloat16 if is8 else t["q"].dtype, device=dev)
     t["lse"] = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
     if with_bwd:
         t["dq"], t["dk"], t["dv"] = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
         t["ws"] = torch.empty(api.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
-    in_bytes = sum(t[n].numel() * t[n].element_size() for n in ("q", "k", "v", "do"))
+    in_bytes = sum(t[n].numel() * t[n].element_size() for n in names)
 
     step = _step_fn(api, t, w, with_bwd)
     clocks = ClockSampler(dev.index)
@@ -329,14 +342,14 @@ def run_ours(args, w):
     status = api.get_status()
 
     # ---------------- end-to-end through the public API: pinned host in, results back
-    host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "do")}
+    host = {n: inp[n].pin_memory() for n in names}
     out_host = {n: torch.empty(t[n].shape, dtype=t[n].dtype).pin_memory()
                 for n in (["o", "lse"] + (["dq", "dk", "dv"] if with_bwd else []))}
     d2h_bytes = sum(x.numel() * x.element_size() for x in out_host.values())
     e2e_steps = max(1, min(args.steps, 20))
 
     def e2e_step():
-        for n in ("q", "k", "v", "do"):
+        for n in names:
             t[n].copy_(host[n], non_blocking=True)
         step()
         for n, x in out_host.items():
@@ -364,6 +377,9 @@ def run_ours(args, w):
     value = whole_job_tflops(world, step_flops, ms)
     e2e_value = whole_job_tflops(world, step_flops, e2e_ms)
     peak, peak_sus, hbm, peak_kind = _peaks()
+    if is8:
+        # e4m3 contraction: the measured bf16 peak times the nominal dense e4m3 / bf16 ratio (2)
+        peak, peak_sus, peak_kind = 2 * peak, 2 * peak_sus, peak_kind + " bf16 x 2 (nominal e4m3/bf16 ratio);"
     fwd_tf = ff / (fwd_ms * 1e-3) / 1e12
     bwd_tf = fb / (bwd_ms * 1e-3) / 1e12 if with_bwd else None
     # dominant kernel: the one with the larger share of the step
@@ -374,18 +390,20 @@ def run_ours(args, w):
     roofline = {"bound": "tensor", "achieved": dom["achieved"], "peak": peak, "unit": "TFLOP/s",
                 "frac": dom["achieved"] / peak, "traffic": measured_traffic(dom["key"], w.name),
                 "kernel": dom["kernel"],
-                "peak_kind": f"{peak_kind} bf16 burst (cuBLAS 8192^3)",
+                "peak_kind": f"{peak_kind} bf16 burst (cuBLAS 8192^3)" if not is8 else f"{peak_kind} burst",
                 "frac_of_sustained": dom["achieved"] / peak_sus,
                 "fwd_alg_bytes": fwd_bytes(w.B, w.H, w.N, w.d)}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                    "H_kv": w.H_kv or w.H, "window": w.window,
                    "parallelism": f"replicas x{world}",
                    "l2": f"not flushed: inputs {in_bytes / 1e6:.0f} MB > L2 {L2_BYTES / 1e6:.0f} MB",
-                   "step": "fa_fwd + fa_bwd" if with_bwd else "fa_fwd only (backward not built)"},
+                   "step": "fa_fwd + fa_bwd" if with_bwd else
+                           ("fa_fwd_e4m3_scaled (the e4m3 path is forward only)" if is8 else
+                            "fa_fwd only (backward not built)")},
         "fwd_tflops": fwd_tf, "fwd_ms": fwd_ms, "bwd_tflops": bwd_tf, "bwd_ms": bwd_ms,
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": roofline,
@@ -402,7 +420,8 @@ def run_ours(args, w):
         line["cpu_baseline"] = {
             "value": cflops / cdt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
             "sample": f"{heads} full heads of {w.name} (forward" + (" + backward" if with_bwd else "")
-                      + f", fp64), {cdt:.1f} s"}
+                      + f", fp64{'; bf16-drawn inputs, the oracle costs the same for any input type' if is8 else ''}),"
+                      f" {cdt:.1f} s"}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

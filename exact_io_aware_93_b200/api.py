@@ -26,18 +26,21 @@ FA_STATUS = {
 }
 
 
+FA_DTYPE = {torch.bfloat16: 0, torch.float16: 1, torch.float8_e4m3fn: 2}
+
+
 class FaProblem(ctypes.Structure):
     """The ``fa_problem`` descriptor of include/fa.h."""
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int), ("N", ctypes.c_int),
                 ("d", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int),
-                ("window", ctypes.c_int)]
+                ("window", ctypes.c_int), ("dtype", ctypes.c_int)]
 
 
 class FaDecodeProblem(ctypes.Structure):
     """The ``fa_decode_problem`` descriptor of include/fa.h."""
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int), ("N_q", ctypes.c_int),
                 ("N_kv", ctypes.c_int), ("d", ctypes.c_int), ("scale", ctypes.c_float),
-                ("causal", ctypes.c_int), ("window", ctypes.c_int)]
+                ("causal", ctypes.c_int), ("window", ctypes.c_int), ("dtype", ctypes.c_int)]
 
 
 class FAError(RuntimeError):
@@ -83,6 +86,8 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
                          i, i, i, i, f, i, vp]
     L.fa_bwd.restype = i
+    L.fa_fwd_e4m3_scaled.argtypes = [ctypes.POINTER(FaProblem), vp, vp, vp, f, f, f, vp, vp, vp]
+    L.fa_fwd_e4m3_scaled.restype = i
     L.fa_decode_workspace_size.argtypes = [ctypes.POINTER(FaDecodeProblem)]
     L.fa_decode_workspace_size.restype = ctypes.c_size_t
     L.fa_decode.argtypes = [ctypes.POINTER(FaDecodeProblem), vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
@@ -101,8 +106,8 @@ def validate_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
             raise TypeError(f"{name} must be a torch.Tensor")
         if t.dim() != 4:
             raise ValueError(f"{name} must be [batch, seq_len, num_heads, head_dim], got {tuple(t.shape)}")
-        if t.dtype != torch.bfloat16:
-            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if t.dtype not in FA_DTYPE:
+            raise TypeError(f"{name} must be bfloat16, float16 or float8_e4m3fn, got {t.dtype}")
         if not t.is_cuda:
             raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
         if not t.is_contiguous():
@@ -120,26 +125,29 @@ def validate_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
         raise ValueError(f"query and key sequence lengths must match: {q.shape[1]}, {k.shape[1]}")
     if not (q.device == k.device == v.device):
         raise ValueError("q, k, v must be on the same device")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError(f"q, k, v must share one dtype, got {q.dtype}, {k.dtype}, {v.dtype}")
 
 
 def problem(q: torch.Tensor, k: torch.Tensor, causal: bool, scale: float | None,
             window: int | None) -> FaProblem:
     B, N, H, d = q.shape
     return FaProblem(B, H, k.shape[2], N, d, 1.0 / math.sqrt(d) if scale is None else float(scale),
-                     int(bool(causal)), -1 if window is None else int(window))
+                     int(bool(causal)), -1 if window is None else int(window), FA_DTYPE[q.dtype])
 
 
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         scale: float | None = None, out: torch.Tensor | None = None,
         lse: torch.Tensor | None = None, window: int | None = None):
-    """(O [B, N, H, d] bf16, LSE [B, H, N] fp32) of exact attention via ``fa_fwd_ex``.
+    """(O [B, N, H, d] in q's dtype, LSE [B, H, N] fp32) of exact attention via ``fa_fwd_ex``.
 
     k and v may have fewer heads than q (grouped-query attention); ``window`` (causal only)
     limits query i to keys i - window .. i."""
     validate_inputs(q, k, v)
     B, N, H, d = q.shape
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=torch.bfloat16 if q.dtype == torch.float8_e4m3fn else q.dtype,
+                          device=q.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     p = problem(q, k, causal, scale, window)
@@ -147,6 +155,26 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
                          lse.data_ptr(), _stream_ptr(q))
     if st != 0:
         raise FAError(st, "fa_fwd_ex")
+    return out, lse
+
+
+def fwd_e4m3(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_descale: float, k_descale: float,
+             v_descale: float, causal: bool = False, scale: float | None = None, out: torch.Tensor | None = None,
+             lse: torch.Tensor | None = None, window: int | None = None):
+    """(O [B, N, H, d] bf16, LSE [B, H, N] fp32) of attention over the values ``codes * descale``
+    of fp8 e4m3 inputs (torch.float8_e4m3fn), via ``fa_fwd_e4m3_scaled`` (d = 128)."""
+    validate_inputs(q, k, v)
+    if q.dtype != torch.float8_e4m3fn:
+        raise TypeError("fwd_e4m3 takes float8_e4m3fn codes")
+    B, N, H, d = q.shape
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    p = problem(q, k, causal, scale, window)
+    st = lib().fa_fwd_e4m3_scaled(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                  float(q_descale), float(k_descale), float(v_descale), out.data_ptr(),
+                                  lse.data_ptr(), _stream_ptr(q))
+    if st != 0:
+        raise FAError(st, "fa_fwd_e4m3_scaled")
     return out, lse
 
 
@@ -162,8 +190,8 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, do: 
     """(dQ, dK, dV) of L = sum(O * dO) via ``fa_bwd_ex`` (score tiles recomputed from LSE)."""
     validate_inputs(q, k, v)
     for name, t in (("o", o), ("do", do)):
-        if t.shape != q.shape or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device != q.device:
-            raise ValueError(f"{name} must be a contiguous bf16 tensor shaped like q")
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name} must be a contiguous tensor shaped like q, of q's dtype")
     B, N, H, d = q.shape
     if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
@@ -188,7 +216,7 @@ def decode_problem(q: torch.Tensor, k_cache: torch.Tensor, causal: bool, scale: 
     B, n_q, H, d = q.shape
     return FaDecodeProblem(B, H, k_cache.shape[2], n_q, k_cache.shape[1], d,
                            1.0 / math.sqrt(d) if scale is None else float(scale), int(bool(causal)),
-                           -1 if window is None else int(window))
+                           -1 if window is None else int(window), FA_DTYPE.get(q.dtype, -1))
 
 
 def decode_workspace_size(q: torch.Tensor, k_cache: torch.Tensor, causal: bool = True,
@@ -201,15 +229,15 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
            seqlens: torch.Tensor | None = None, causal: bool = True, scale: float | None = None,
            out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
            workspace: torch.Tensor | None = None, window: int | None = None):
-    """(O [B, N_q, H, d] bf16, LSE [B, H, N_q] fp32) of N_q new queries per sequence against a
+    """(O [B, N_q, H, d] in q's dtype, LSE [B, H, N_q] fp32) of N_q new queries per sequence against a
     key/value cache ``[B, N_kv, H_kv, d]`` via ``fa_decode``.
 
     ``seqlens`` (int32 [B] on the device, or None for full caches) gives each sequence's cached
     length; with ``causal`` the queries are the last N_q positions of each sequence: query i
     of sequence b stands at position seqlens[b] - N_q + i."""
     for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
-        if not isinstance(t, torch.Tensor) or t.dim() != 4 or t.dtype != torch.bfloat16:
-            raise ValueError(f"{name} must be a 4-d bfloat16 tensor")
+        if not isinstance(t, torch.Tensor) or t.dim() != 4 or t.dtype not in FA_DTYPE or t.dtype != q.dtype:
+            raise ValueError(f"{name} must be a 4-d bfloat16 or float16 tensor of q's dtype")
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor (no CPU path)")
     B, n_q, H, d = q.shape

@@ -25,9 +25,9 @@ struct DeviceInfo {
   bool ok = false;
   int sm_count = 0;
   int* status = nullptr;
-  bool fwd_attr[2][2] = {{false, false}, {false, false}};  // [d==128][causal]
-  bool bwd_attr[2][2] = {{false, false}, {false, false}};
-  bool dec_attr[2] = {false, false};  // [d==128]
+  bool fwd_attr[3][2][2] = {};  // [element type][d==128][causal]
+  bool bwd_attr[2][2][2] = {};
+  bool dec_attr[2][2] = {};     // [fp16][d==128]
 };
 DeviceInfo g_dev[kMaxDevices];
 
@@ -74,6 +74,8 @@ fa_status current_device(DeviceInfo** out) {
 }
 
 fa_status check_problem(const fa_problem& p) {
+  if (p.dtype != FA_DTYPE_BF16 && p.dtype != FA_DTYPE_F16 && p.dtype != FA_DTYPE_E4M3) return FA_ERR_UNSUPPORTED;
+  if (p.dtype == FA_DTYPE_E4M3 && p.d != 128) return FA_ERR_UNSUPPORTED;
   if (p.H_kv < 1 || p.H_kv > p.H || (p.H_kv >= 1 && p.H % p.H_kv != 0)) return FA_ERR_INVALID_ARG;
   if (p.window < -1 || (p.window >= 0 && p.causal != 1)) return FA_ERR_INVALID_ARG;
   return FA_OK;
@@ -92,12 +94,14 @@ fa_status check_common(int B, int H, int N, int d, float scale, int causal) {
   return FA_OK;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, fa::Elem E>
 fa_status launch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o,
-                     float* lse, int B, int H, int H_kv, int N, int window, float scale, cudaStream_t stream) {
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
-  const int smem = static_cast<int>(sizeof(fa::FwdSmem<D>)) + 1024;
-  bool& attr = di.fwd_attr[D == 128][CAUSAL];
+                     float* lse, int B, int H, int H_kv, int N, int window, float scale, cudaStream_t stream,
+                     float out_scale = 1.0f) {
+  using T = typename fa::FwdOut<E>::T;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, E>;
+  const int smem = static_cast<int>(sizeof(fa::FwdSmem<D, E>)) + 1024;
+  bool& attr = di.fwd_attr[static_cast<int>(E)][D == 128][CAUSAL];
   if (!attr) {
     if (!launch_regs_ok(kern, fa::kLaunchRegs) ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
@@ -110,8 +114,8 @@ fa_status launch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   const long long tiles = static_cast<long long>(B) * H * ((nkb + 1) / 2);
   const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
   const float scale_log2 = scale * 1.4426950408889634f;
-  kern<<<grid, fa::kFwdThreads, smem, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, B, H, H_kv, N,
-                                                 window, scale_log2, di.status);
+  kern<<<grid, fa::kFwdThreads, smem, stream>>>(mq, mk, mv, static_cast<T*>(o), lse, B, H, H_kv, N, window,
+                                                 scale_log2, out_scale, di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
 }
@@ -124,26 +128,26 @@ size_t bwd_ws_bytes(int B, int H, int N, int d) {
   return bh * static_cast<size_t>(N) * static_cast<size_t>(d) * 4 + 2 * bh * npad * 4;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, fa::Elem E>
 fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& mdo, const void* o, const void* dO, const float* lse, void* dq, void* dk,
                      void* dv, void* ws, int B, int H, int H_kv, int N, int window, float scale,
                      cudaStream_t stream) {
+  using T = typename fa::ElemOps<E>::T;
   const int64_t rows = static_cast<int64_t>(B) * H * N;
   const int64_t prows = static_cast<int64_t>(B) * H * ((N + 127) / 128 * 128);
   float* dq_acc = static_cast<float*>(ws);
   float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + rows * D * 4);
   float* lse2 = dsum + prows;
   const unsigned pre_blocks = static_cast<unsigned>((prows * (D / 8) + 255) / 256);
-  fa::fa_bwd_pre_kernel<D><<<pre_blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                           static_cast<const __nv_bfloat16*>(dO), lse, dsum, lse2,
-                                                           dq_acc, B, H, N);
+  fa::fa_bwd_pre_kernel<D, E><<<pre_blocks, 256, 0, stream>>>(static_cast<const T*>(o), static_cast<const T*>(dO),
+                                                              lse, dsum, lse2, dq_acc, B, H, N);
   const int64_t ew_threads = rows * (D / 8);
   const unsigned ew_blocks = static_cast<unsigned>((ew_threads + 255) / 256);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
-  auto kern = fa::fa_bwd_main_kernel<D, CAUSAL>;
+  auto kern = fa::fa_bwd_main_kernel<D, CAUSAL, E>;
   const int smem = static_cast<int>(sizeof(fa::BwdSmem<D>));
-  bool& attr = di.bwd_attr[D == 128][CAUSAL];
+  bool& attr = di.bwd_attr[E == fa::Elem::kF16][D == 128][CAUSAL];
   if (!attr) {
     if (!launch_regs_ok(kern, fa::kBwdLaunchRegs) ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
@@ -153,15 +157,61 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
     attr = true;
   }
   const int nkb = (N + 127) / 128;
-  kern<<<B * H_kv * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, lse2, dsum, dq_acc,
-                                                           static_cast<__nv_bfloat16*>(dk),
-                                                           static_cast<__nv_bfloat16*>(dv), B, H, H_kv, N, window,
-                                                           scale, di.status);
+  kern<<<B * H_kv * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, lse2, dsum, dq_acc, static_cast<T*>(dk),
+                                                           static_cast<T*>(dv), B, H, H_kv, N, window, scale,
+                                                           di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
-  fa::fa_bwd_post_kernel<D><<<ew_blocks, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), B, H, N,
-                                                           scale);
+  fa::fa_bwd_post_kernel<D, E><<<ew_blocks, 256, 0, stream>>>(dq_acc, static_cast<T*>(dq), B, H, N, scale);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
+}
+
+template <fa::Elem E>
+fa_status dispatch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o,
+                       float* lse, const fa_problem& p, cudaStream_t s) {
+  const int w = p.window;
+  if (p.d == 128)
+    return p.causal ? launch_fwd<128, true, E>(di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s)
+                    : launch_fwd<128, false, E>(di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s);
+  return p.causal ? launch_fwd<64, true, E>(di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s)
+                  : launch_fwd<64, false, E>(di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s);
+}
+
+fa_status dispatch_fwd_e4m3(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                           void* o, float* lse, const fa_problem& p, float out_scale, cudaStream_t s) {
+  constexpr fa::Elem E = fa::Elem::kE4M3;
+  const int w = p.window;
+  return p.causal ? launch_fwd<128, true, E>(di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s, out_scale)
+                  : launch_fwd<128, false, E>(di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s, out_scale);
+}
+
+fa::MapElem map_elem(int dtype) {
+  return dtype == FA_DTYPE_F16 ? fa::MapElem::kF16 : (dtype == FA_DTYPE_E4M3 ? fa::MapElem::kE4M3 : fa::MapElem::kBf16);
+}
+
+struct BwdPtrs {
+  const void* o;
+  const void* dO;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  void* ws;
+};
+
+template <fa::Elem E>
+fa_status dispatch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const CUtensorMap& mdo, const BwdPtrs& x, const fa_problem& p, cudaStream_t s) {
+  const int B = p.B, H = p.H, H_kv = p.H_kv, N = p.N, w = p.window;
+  if (p.d == 128)
+    return p.causal ? launch_bwd<128, true, E>(di, mq, mk, mv, mdo, x.o, x.dO, x.lse, x.dq, x.dk, x.dv, x.ws, B, H,
+                                               H_kv, N, w, p.scale, s)
+                    : launch_bwd<128, false, E>(di, mq, mk, mv, mdo, x.o, x.dO, x.lse, x.dq, x.dk, x.dv, x.ws, B, H,
+                                                H_kv, N, w, p.scale, s);
+  return p.causal ? launch_bwd<64, true, E>(di, mq, mk, mv, mdo, x.o, x.dO, x.lse, x.dq, x.dk, x.dv, x.ws, B, H,
+                                            H_kv, N, w, p.scale, s)
+                  : launch_bwd<64, false, E>(di, mq, mk, mv, mdo, x.o, x.dO, x.lse, x.dq, x.dk, x.dv, x.ws, B, H,
+                                             H_kv, N, w, p.scale, s);
 }
 
 // ---------------------------------------------------------------- decoding
@@ -172,6 +222,7 @@ fa_status check_decode(const fa_decode_problem& p) {
   if (p.causal != 0 && p.causal != 1) return FA_ERR_INVALID_ARG;
   if (p.window < -1 || (p.window >= 0 && p.causal != 1)) return FA_ERR_INVALID_ARG;
   if (p.d != 64 && p.d != 128) return FA_ERR_UNSUPPORTED;
+  if (p.dtype != FA_DTYPE_BF16 && p.dtype != FA_DTYPE_F16) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(p.H / p.H_kv) * p.N_q > fa::kDecMaxRows) return FA_ERR_UNSUPPORTED;
   // tile counts, tile starts and element offsets stay in range
   const long long tiles = static_cast<long long>(p.B) * p.H_kv * ((static_cast<long long>(p.N_kv) + 127) / 128);
@@ -201,13 +252,13 @@ DecLayout dec_layout(const fa_decode_problem& p, int grid) {
   return L;
 }
 
-template <int D>
+template <int D, fa::Elem E>
 fa_status launch_decode(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         const fa_decode_problem& p, const int* seqlens, void* o, float* lse, void* ws,
                         cudaStream_t stream) {
-  auto kern = fa::fa_decode_kernel<D>;
+  auto kern = fa::fa_decode_kernel<D, E>;
   const int smem = static_cast<int>(sizeof(fa::DecSmem<D>)) + 1024;
-  bool& attr = di.dec_attr[D == 128];
+  bool& attr = di.dec_attr[E == fa::Elem::kF16][D == 128];
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
       cudaGetLastError();
@@ -220,7 +271,7 @@ fa_status launch_decode(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap
   uint8_t* w = static_cast<uint8_t*>(ws);
   fa::DecArgs a;
   a.seqlens = seqlens;
-  a.out = static_cast<__nv_bfloat16*>(o);
+  a.out = o;
   a.lse = lse;
   a.meta = reinterpret_cast<int*>(w + L.meta);
   a.part_lse = reinterpret_cast<float*>(w + L.part_lse);
@@ -235,7 +286,7 @@ fa_status launch_decode(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap
   a.scale_log2 = p.scale * 1.4426950408889634f;
   kern<<<grid, fa::kDecThreads, smem, stream>>>(mq, mk, mv, a, di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
-  fa::fa_decode_merge_kernel<D><<<p.B * p.H_kv, 128, 0, stream>>>(a);
+  fa::fa_decode_merge_kernel<D, E><<<p.B * p.H_kv, 128, 0, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
 }
@@ -298,7 +349,7 @@ fa_status noalloc_scratch(void** out) {
 
 extern "C" {
 
-int fa_abi_version(void) { return 3; }
+int fa_abi_version(void) { return 4; }
 
 const char* fa_status_string(int s) {
   switch (s) {
@@ -314,35 +365,56 @@ const char* fa_status_string(int s) {
   }
 }
 
+static fa_status fwd_common(const fa_problem* problem, const void* q, const void* k, const void* v, void* o,
+                            float* lse, float q_descale, float k_descale, float v_descale, void* stream);
+
 fa_status fa_fwd_ex(const fa_problem* problem, const void* q, const void* k, const void* v, void* o, float* lse,
                     void* stream) {
+  return fwd_common(problem, q, k, v, o, lse, 1.0f, 1.0f, 1.0f, stream);
+}
+
+fa_status fa_fwd_e4m3_scaled(const fa_problem* problem, const void* q, const void* k, const void* v,
+                             float q_descale, float k_descale, float v_descale, void* o, float* lse, void* stream) {
+  if (!problem) return FA_ERR_INVALID_ARG;
+  if (problem->dtype != FA_DTYPE_E4M3) return FA_ERR_INVALID_ARG;
+  return fwd_common(problem, q, k, v, o, lse, q_descale, k_descale, v_descale, stream);
+}
+
+static fa_status fwd_common(const fa_problem* problem, const void* q, const void* k, const void* v, void* o,
+                            float* lse, float q_descale, float k_descale, float v_descale, void* stream) {
   if (!problem || !q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   const fa_problem p = *problem;
   fa_status st = check_common(p.B, p.H, p.N, p.d, p.scale, p.causal);
   if (st != FA_OK) return st;
   st = check_problem(p);
   if (st != FA_OK) return st;
+  for (const float x : {q_descale, k_descale, v_descale})
+    if (!(x > 0.0f) || !isfinite(x)) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGNMENT;
   DeviceInfo* di = nullptr;
   st = current_device(&di);
   if (st != FA_OK) return st;
   CUtensorMap mq, mk, mv;
-  if (!fa::make_bshd_map(&mq, q, p.B, p.N, p.H, p.d, 128) || !fa::make_bshd_map(&mk, k, p.B, p.N, p.H_kv, p.d, 128) ||
-      !fa::make_bshd_map(&mv, v, p.B, p.N, p.H_kv, p.d, 128))
+  const fa::MapElem me = map_elem(p.dtype);
+  if (!fa::make_bshd_map(&mq, q, p.B, p.N, p.H, p.d, 128, me) ||
+      !fa::make_bshd_map(&mk, k, p.B, p.N, p.H_kv, p.d, 128, me) ||
+      !fa::make_bshd_map(&mv, v, p.B, p.N, p.H_kv, p.d, 128, me))
     return FA_ERR_LAUNCH;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int w = p.window;
-  if (p.d == 128)
-    return p.causal ? launch_fwd<128, true>(*di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s)
-                    : launch_fwd<128, false>(*di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s);
-  return p.causal ? launch_fwd<64, true>(*di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s)
-                  : launch_fwd<64, false>(*di, mq, mk, mv, o, lse, p.B, p.H, p.H_kv, p.N, w, p.scale, s);
+  if (p.dtype == FA_DTYPE_E4M3) {
+    // the dequantisation factors of Q and K scale the scores; V's scales the output
+    fa_problem pe = p;
+    pe.scale = p.scale * q_descale * k_descale;
+    return dispatch_fwd_e4m3(*di, mq, mk, mv, o, lse, pe, v_descale, s);
+  }
+  return p.dtype == FA_DTYPE_F16 ? dispatch_fwd<fa::Elem::kF16>(*di, mq, mk, mv, o, lse, p, s)
+                                 : dispatch_fwd<fa::Elem::kBf16>(*di, mq, mk, mv, o, lse, p, s);
 }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  float scale, int causal, void* stream) {
-  const fa_problem p{B, H, H, N, d, scale, causal, -1};
+  const fa_problem p{B, H, H, N, d, scale, causal, -1, FA_DTYPE_BF16};
   return fa_fwd_ex(&p, q, k, v, o, lse, stream);
 }
 
@@ -361,12 +433,13 @@ fa_status fa_bwd_ex(const fa_problem* problem, const void* q, const void* k, con
                     size_t workspace_bytes, void* stream) {
   if (!problem || !q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   const fa_problem p = *problem;
-  const int B = p.B, H = p.H, H_kv = p.H_kv, N = p.N, d = p.d, causal = p.causal, window = p.window;
+  const int B = p.B, H = p.H, H_kv = p.H_kv, N = p.N, d = p.d, causal = p.causal;
   const float scale = p.scale;
   fa_status st = check_common(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
   st = check_problem(p);
   if (st != FA_OK) return st;
+  if (p.dtype == FA_DTYPE_E4M3) return FA_ERR_UNSUPPORTED;  // the e4m3 path is forward only
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
       !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGNMENT;
@@ -377,25 +450,21 @@ fa_status fa_bwd_ex(const fa_problem* problem, const void* q, const void* k, con
   st = current_device(&di);
   if (st != FA_OK) return st;
   CUtensorMap mq, mk, mv, mdo;
-  if (!fa::make_bshd_map(&mq, q, B, N, H, d, 128) || !fa::make_bshd_map(&mk, k, B, N, H_kv, d, 128) ||
-      !fa::make_bshd_map(&mv, v, B, N, H_kv, d, 128) || !fa::make_bshd_map(&mdo, dO, B, N, H, d, 128))
+  const bool f16 = p.dtype == FA_DTYPE_F16;
+  const fa::MapElem me = map_elem(p.dtype);
+  if (!fa::make_bshd_map(&mq, q, B, N, H, d, 128, me) || !fa::make_bshd_map(&mk, k, B, N, H_kv, d, 128, me) ||
+      !fa::make_bshd_map(&mv, v, B, N, H_kv, d, 128, me) || !fa::make_bshd_map(&mdo, dO, B, N, H, d, 128, me))
     return FA_ERR_LAUNCH;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 128)
-    return causal ? launch_bwd<128, true>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, H_kv, N,
-                                          window, scale, s)
-                  : launch_bwd<128, false>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, H_kv, N,
-                                           window, scale, s);
-  return causal ? launch_bwd<64, true>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, H_kv, N,
-                                       window, scale, s)
-                : launch_bwd<64, false>(*di, mq, mk, mv, mdo, o, dO, lse, dq, dk, dv, workspace, B, H, H_kv, N,
-                                        window, scale, s);
+  const BwdPtrs ptr{o, dO, lse, dq, dk, dv, workspace};
+  return f16 ? dispatch_bwd<fa::Elem::kF16>(*di, mq, mk, mv, mdo, ptr, p, s)
+             : dispatch_bwd<fa::Elem::kBf16>(*di, mq, mk, mv, mdo, ptr, p, s);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
                  float scale, int causal, void* stream) {
-  const fa_problem p{B, H, H, N, d, scale, causal, -1};
+  const fa_problem p{B, H, H, N, d, scale, causal, -1, FA_DTYPE_BF16};
   return fa_bwd_ex(&p, q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, stream);
 }
 
@@ -436,13 +505,18 @@ fa_status fa_decode(const fa_decode_problem* problem, const void* q, const void*
   if (!aligned(workspace, 256)) return FA_ERR_ALIGNMENT;
   const int G = p.H / p.H_kv;
   CUtensorMap mq, mk, mv;
-  if (!fa::make_decode_q_map(&mq, q, p.B, p.N_q, p.H, p.d, G) ||
-      !fa::make_bshd_map(&mk, k_cache, p.B, p.N_kv, p.H_kv, p.d, 128) ||
-      !fa::make_bshd_map(&mv, v_cache, p.B, p.N_kv, p.H_kv, p.d, 128))
+  const bool f16 = p.dtype == FA_DTYPE_F16;
+  const fa::MapElem me = map_elem(p.dtype);
+  if (!fa::make_decode_q_map(&mq, q, p.B, p.N_q, p.H, p.d, G, me) ||
+      !fa::make_bshd_map(&mk, k_cache, p.B, p.N_kv, p.H_kv, p.d, 128, me) ||
+      !fa::make_bshd_map(&mv, v_cache, p.B, p.N_kv, p.H_kv, p.d, 128, me))
     return FA_ERR_LAUNCH;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (p.d == 128) return launch_decode<128>(*di, mq, mk, mv, p, seqlens, o, lse, workspace, s);
-  return launch_decode<64>(*di, mq, mk, mv, p, seqlens, o, lse, workspace, s);
+  if (f16)
+    return p.d == 128 ? launch_decode<128, fa::Elem::kF16>(*di, mq, mk, mv, p, seqlens, o, lse, workspace, s)
+                      : launch_decode<64, fa::Elem::kF16>(*di, mq, mk, mv, p, seqlens, o, lse, workspace, s);
+  return p.d == 128 ? launch_decode<128, fa::Elem::kBf16>(*di, mq, mk, mv, p, seqlens, o, lse, workspace, s)
+                    : launch_decode<64, fa::Elem::kBf16>(*di, mq, mk, mv, p, seqlens, o, lse, workspace, s);
 }
 
 fa_status fa_selftest_wait_timeout(unsigned int timeout_us, void* stream) {

@@ -100,9 +100,9 @@ struct __align__(1024) BwdSmem {
 // [B*H, Npad] with Npad = N rounded up to 128; rows n in [N, Npad) get D = 0 and
 // LSE2 = +inf, so every 128-row block is a full, 16-byte-aligned 512-byte run and its
 // padded queries have P = 0.  One group of D/8 threads per row, 16-byte loads.
-template <int D>
-__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
-                                                         const __nv_bfloat16* __restrict__ dout,
+template <int D, Elem E = Elem::kBf16>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const typename ElemOps<E>::T* __restrict__ o,
+                                                         const typename ElemOps<E>::T* __restrict__ dout,
                                                          const float* __restrict__ lse,
                                                          float* __restrict__ dsum, float* __restrict__ lse2,
                                                          float* __restrict__ dq_acc, int B, int H, int N) {
@@ -120,12 +120,12 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
     const int64_t off = ((static_cast<int64_t>(b) * N + n) * H + h) * D + part * 8;
     const uint4 ov = *reinterpret_cast<const uint4*>(o + off);
     const uint4 dv = *reinterpret_cast<const uint4*>(dout + off);
-    const __nv_bfloat162* op = reinterpret_cast<const __nv_bfloat162*>(&ov);
-    const __nv_bfloat162* dp = reinterpret_cast<const __nv_bfloat162*>(&dv);
+    const uint32_t* op = reinterpret_cast<const uint32_t*>(&ov);
+    const uint32_t* dp = reinterpret_cast<const uint32_t*>(&dv);
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
-      const float2 a = __bfloat1622float2(op[x]);
-      const float2 c = __bfloat1622float2(dp[x]);
+      const float2 a = ElemOps<E>::unpack(op[x]);
+      const float2 c = ElemOps<E>::unpack(dp[x]);
       acc = fmaf(a.x, c.x, acc);
       acc = fmaf(a.y, c.y, acc);
     }
@@ -142,10 +142,10 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
 }
 
 // ---------------------------------------------------------------- post
-// dQ[b,n,h,:] = bf16(scale * acc[b,h,n,:]), 8 elements per thread.
-template <int D>
+// dQ[b,n,h,:] = (scale * acc[b,h,n,:]) in the input type, 8 elements per thread.
+template <int D, Elem E = Elem::kBf16>
 __global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restrict__ dq_acc,
-                                                          __nv_bfloat16* __restrict__ dq, int B, int H, int N,
+                                                          typename ElemOps<E>::T* __restrict__ dq, int B, int H, int N,
                                                           float scale) {
   constexpr int TPR = D / 8;
   const int64_t rows = static_cast<int64_t>(B) * H * N;
@@ -158,10 +158,10 @@ __global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restric
   const float4* a = reinterpret_cast<const float4*>(dq_acc + row * D + part * 8);
   const float4 a0 = a[0], a1 = a[1];
   uint4 r;
-  r.x = pack_bf16x2(a0.x * scale, a0.y * scale);
-  r.y = pack_bf16x2(a0.z * scale, a0.w * scale);
-  r.z = pack_bf16x2(a1.x * scale, a1.y * scale);
-  r.w = pack_bf16x2(a1.z * scale, a1.w * scale);
+  r.x = ElemOps<E>::pack(a0.x * scale, a0.y * scale);
+  r.y = ElemOps<E>::pack(a0.z * scale, a0.w * scale);
+  r.z = ElemOps<E>::pack(a1.x * scale, a1.y * scale);
+  r.w = ElemOps<E>::pack(a1.z * scale, a1.w * scale);
   *reinterpret_cast<uint4*>(dq + ((static_cast<int64_t>(b) * N + n) * H + h) * D + part * 8) = r;
 }
 
@@ -179,7 +179,7 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 // qhi past the end of a sliding window);
 // returns the 16 bf16 pairs.  One branch per chunk instead of one per element keeps the
 // unrolled loop a single basic block the compiler can interleave.
-template <bool MASKED>
+template <bool MASKED, Elem E = Elem::kBf16>
 __device__ __forceinline__ void bwd_p_chunk(const uint32_t (&sv)[32], const float* lse2, float2 sl2, int q0,
                                             bool key_ok, int qlim, int qhi, uint32_t* pk) {
   float4 l4[8];
@@ -200,18 +200,19 @@ __device__ __forceinline__ void bwd_p_chunk(const uint32_t (&sv)[32], const floa
       p2 = (key_ok && ql + 2 >= qlim && ql + 2 <= qhi) ? p2 : 0.f;
       p3 = (key_ok && ql + 3 >= qlim && ql + 3 <= qhi) ? p3 : 0.f;
     }
-    pk[x / 2] = pack_bf16x2(p0, p1);
-    pk[x / 2 + 1] = pack_bf16x2(p2, p3);
+    pk[x / 2] = ElemOps<E>::pack(p0, p1);
+    pk[x / 2 + 1] = ElemOps<E>::pack(p2, p3);
   }
 }
 
 // ---------------------------------------------------------------- main
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, Elem E = Elem::kBf16>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                        const float* __restrict__ lse2g, const float* __restrict__ dsum,
-                       float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                       float* __restrict__ dq_acc, typename ElemOps<E>::T* __restrict__ dk,
+                       typename ElemOps<E>::T* __restrict__ dv,
                        int B, int H, int H_kv, int N, int window, float scale, int* status) {
   using Cfg = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -318,9 +319,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const WaitCtx wc{&sm.abort_flag, status, 12};
-      constexpr uint32_t idesc_sdp = idesc_bf16(128, 128, 0, 0);  // K-major x K-major
-      constexpr uint32_t idesc_acc = idesc_bf16(128, D, 0, 1);    // K-major (TMEM or smem) A x MN-major B
-      constexpr uint32_t idesc_dq = idesc_bf16(128, D, 1, 1);     // MN-major A (dS) x MN-major B (K)
+      constexpr uint32_t kT = ElemOps<E>::kMmaType;
+      constexpr uint32_t idesc_sdp = idesc_kind_f16(128, 128, 0, 0, kT);  // K-major x K-major
+      constexpr uint32_t idesc_acc = idesc_kind_f16(128, D, 0, 1, kT);    // K-major (TMEM or smem) A x MN-major B
+      constexpr uint32_t idesc_dq = idesc_kind_f16(128, D, 1, 1, kT);     // MN-major A (dS) x MN-major B (K)
       const uint64_t dk_kmaj = sdesc_sw128(smem_u32(sm.k), 16, 1024);
       const uint64_t dv_kmaj = sdesc_sw128(smem_u32(sm.v), 16, 1024);
       const uint64_t dk_mn = sdesc_sw128(smem_u32(sm.k), Cfg::kChunkBytes, 1024);
@@ -337,7 +339,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       };
       constexpr bool kDqT = (D == 128);  // dQ^T = K^T dS^T: M = d, N = 128 queries
-      constexpr uint32_t idesc_dqt = idesc_bf16(128, 128, 1, 1);
+      constexpr uint32_t idesc_dqt = idesc_kind_f16(128, 128, 1, 1, kT);
       bool ok = mbar_wait(&sm.kv_full, 0, wc) && mbar_wait(&sm.qd_full[0], 0, wc);
       if (ok) {
         tc_fence_after();
@@ -435,9 +437,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_wait_ld();
         uint32_t* pk = pk_all + 16 * c;
         if (masked)
-          bwd_p_chunk<true>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, qhi, pk);
+          bwd_p_chunk<true, E>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, qhi, pk);
         else
-          bwd_p_chunk<false>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, qhi, pk);
+          bwd_p_chunk<false, E>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, qhi, pk);
         tmem_st16(tS + c * 16, pk);  // columns already read
       }
       tmem_wait_st();
@@ -460,14 +462,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int ql = c * 32 + x;
           const float4 d4 = d4s[x / 4];
           const uint32_t pa = pk_all[ql / 2], pb = pk_all[ql / 2 + 1];
-          const float2 a = fmul2(make_float2(__uint_as_float(pa << 16), __uint_as_float(pa & 0xffff0000u)),
+          const float2 a = fmul2(ElemOps<E>::unpack(pa),
                                  fadd2(make_float2(__uint_as_float(dpv[x]), __uint_as_float(dpv[x + 1])),
                                        make_float2(-d4.x, -d4.y)));
-          const float2 b = fmul2(make_float2(__uint_as_float(pb << 16), __uint_as_float(pb & 0xffff0000u)),
+          const float2 b = fmul2(ElemOps<E>::unpack(pb),
                                  fadd2(make_float2(__uint_as_float(dpv[x + 2]), __uint_as_float(dpv[x + 3])),
                                        make_float2(-d4.z, -d4.w)));
-          dsk[x / 2] = pack_bf16x2(a.x, a.y);
-          dsk[x / 2 + 1] = pack_bf16x2(b.x, b.y);
+          dsk[x / 2] = ElemOps<E>::pack(a.x, a.y);
+          dsk[x / 2 + 1] = ElemOps<E>::pack(b.x, b.y);
         }
         // dS into shared memory: row r of the 128-byte-swizzled MN-major layout; the
         // warpgroup's 64 queries are chunk g, queries 32c..32c+31 its 16-byte units 4c..4c+3
@@ -488,7 +490,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const uint32_t tAcc = tbase + (g == 0 ? Cfg::kColDV : Cfg::kColDK) + lane_off;
       const float mul = g == 0 ? 1.0f : scale;
-      __nv_bfloat16* dst = (g == 0 ? dv : dk) + ((static_cast<int64_t>(b) * N + kg) * H_kv + hkv) * D;
+      typename ElemOps<E>::T* dst = (g == 0 ? dv : dk) + ((static_cast<int64_t>(b) * N + kg) * H_kv + hkv) * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t a[32];
@@ -499,10 +501,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int x = 0; x < 4; ++x)
             pv[x] = make_uint4(
-                pack_bf16x2(__uint_as_float(a[8 * x]) * mul, __uint_as_float(a[8 * x + 1]) * mul),
-                pack_bf16x2(__uint_as_float(a[8 * x + 2]) * mul, __uint_as_float(a[8 * x + 3]) * mul),
-                pack_bf16x2(__uint_as_float(a[8 * x + 4]) * mul, __uint_as_float(a[8 * x + 5]) * mul),
-                pack_bf16x2(__uint_as_float(a[8 * x + 6]) * mul, __uint_as_float(a[8 * x + 7]) * mul));
+                ElemOps<E>::pack(__uint_as_float(a[8 * x]) * mul, __uint_as_float(a[8 * x + 1]) * mul),
+                ElemOps<E>::pack(__uint_as_float(a[8 * x + 2]) * mul, __uint_as_float(a[8 * x + 3]) * mul),
+                ElemOps<E>::pack(__uint_as_float(a[8 * x + 4]) * mul, __uint_as_float(a[8 * x + 5]) * mul),
+                ElemOps<E>::pack(__uint_as_float(a[8 * x + 6]) * mul, __uint_as_float(a[8 * x + 7]) * mul));
         }
       }
     }

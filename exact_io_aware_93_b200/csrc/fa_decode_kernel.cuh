@@ -88,7 +88,7 @@ struct __align__(1024) DecSmem {
 
 struct DecArgs {
   const int* seqlens;      // [B] cached length of each sequence, or null: all N_kv
-  __nv_bfloat16* out;      // [B, N_q, H, D]
+  void* out;               // [B, N_q, H, D], bf16 or fp16
   float* lse;              // [B, H, N_q]
   int* meta;               // [2 + B]: total tiles, tiles per CTA, per-sequence tile prefix
   float* part_lse;         // [slots, M, 2]: natural-log sums of l and of lr of a segment
@@ -196,7 +196,7 @@ struct DecWalk {
   }
 };
 
-template <int D>
+template <int D, Elem E = Elem::kBf16>
 __global__ void __launch_bounds__(kDecThreads, 1)
     fa_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const DecArgs a, int* status) {
@@ -289,8 +289,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // waits; lane 0 issues; the warp zeroes stale value rows)
     const WaitCtx wc{&sm.abort_flag, status, 22};
     const bool leader = lane == 0;
-    constexpr uint32_t idesc_s = idesc_bf16(128, kBN, 0, 0);  // Q, K both K-major
-    constexpr uint32_t idesc_o = idesc_bf16(128, D, 0, 1);    // P from TMEM, V MN-major
+    constexpr uint32_t idesc_s = idesc_kind_f16(128, kBN, 0, 0, ElemOps<E>::kMmaType);  // Q, K K-major
+    constexpr uint32_t idesc_o = idesc_kind_f16(128, D, 0, 1, ElemOps<E>::kMmaType);    // P in TMEM, V MN-major
     const uint32_t kv_addr0 = smem_u32(sm.kv[0]);
     const uint64_t dq0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
     const uint64_t dq1 = sdesc_sw128(smem_u32(sm.q[1]), 16, 1024);
@@ -478,9 +478,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         uint32_t p[kBN / 2];
         const float m_use = mc == -INFINITY ? 0.f : mc;
         if (masked)
-          softmax_row<false>(sv, p, a.scale_log2, m_use, lc, lrc);
+          softmax_row<false, E>(sv, p, a.scale_log2, m_use, lc, lrc);
         else
-          softmax_row<true>(sv, p, a.scale_log2, m_use, lc, lrc);
+          softmax_row<true, E>(sv, p, a.scale_log2, m_use, lc, lrc);
         tmem_st32(tS + 0, p);
         tmem_st32(tS + 32, p + 32);
         tmem_wait_st();
@@ -533,11 +533,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           v[x] = (a0 * __uint_as_float(o0[x]) + (has1 ? a1 * __uint_as_float(o1[x]) : 0.f)) * inv;
         if (real) {
           if (s.whole) {
-            uint4* dst = reinterpret_cast<uint4*>(a.out + ((static_cast<int64_t>(b) * a.N_q + iq) * a.H + h) * D + c);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<typename ElemOps<E>::T*>(a.out) +
+                                                  ((static_cast<int64_t>(b) * a.N_q + iq) * a.H + h) * D + c);
 #pragma unroll
             for (int x = 0; x < 4; ++x)
-              dst[x] = make_uint4(pack_bf16x2(v[8 * x], v[8 * x + 1]), pack_bf16x2(v[8 * x + 2], v[8 * x + 3]),
-                                  pack_bf16x2(v[8 * x + 4], v[8 * x + 5]), pack_bf16x2(v[8 * x + 6], v[8 * x + 7]));
+              dst[x] = make_uint4(ElemOps<E>::pack(v[8 * x], v[8 * x + 1]), ElemOps<E>::pack(v[8 * x + 2], v[8 * x + 3]),
+                                  ElemOps<E>::pack(v[8 * x + 4], v[8 * x + 5]),
+                                  ElemOps<E>::pack(v[8 * x + 6], v[8 * x + 7]));
           } else {
             float4* dst = reinterpret_cast<float4*>(a.part_o + (slot * M + r) * D + c);
 #pragma unroll
@@ -570,8 +572,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 // the same convex combination one CTA would have formed.  Pairs that one CTA covered were
 // written by it; pairs with no key (empty cache) get O = 0, LSE = -inf.  One block of four
 // warps per pair, one warp per row.
-template <int D>
+template <int D, Elem E = Elem::kBf16>
 __global__ void __launch_bounds__(128) fa_decode_merge_kernel(const DecArgs a) {
+  using T = typename ElemOps<E>::T;
   constexpr unsigned kFull = 0xffffffffu;
   const int p = blockIdx.x;
   const int b = p / a.H_kv;
@@ -584,8 +587,8 @@ __global__ void __launch_bounds__(128) fa_decode_merge_kernel(const DecArgs a) {
   if (q.T == 0) {
     for (int r = warp; r < M; r += 4) {
       const int iq = r / G, h = kvh * G + (r - iq * G);
-      __nv_bfloat16* orow = a.out + ((static_cast<int64_t>(b) * a.N_q + iq) * a.H + h) * D;
-      for (int c = lane; c < D; c += 32) orow[c] = __float2bfloat16(0.f);
+      T* orow = static_cast<T*>(a.out) + ((static_cast<int64_t>(b) * a.N_q + iq) * a.H + h) * D;
+      for (int c = lane; c < D; c += 32) orow[c] = ElemOps<E>::one(0.f);
       if (lane == 0) a.lse[(static_cast<int64_t>(b) * a.H + h) * a.N_q + iq] = -INFINITY;
     }
     return;
@@ -637,9 +640,9 @@ __global__ void __launch_bounds__(128) fa_decode_merge_kernel(const DecArgs a) {
       }
     }
     const int iq = r / G, h = kvh * G + (r - iq * G);
-    __nv_bfloat16* orow = a.out + ((static_cast<int64_t>(b) * a.N_q + iq) * a.H + h) * D;
+    T* orow = static_cast<T*>(a.out) + ((static_cast<int64_t>(b) * a.N_q + iq) * a.H + h) * D;
 #pragma unroll
-    for (int j = 0; j < D / 32; ++j) orow[lane + 32 * j] = __float2bfloat16(acc[j]);
+    for (int j = 0; j < D / 32; ++j) orow[lane + 32 * j] = ElemOps<E>::one(acc[j]);
     if (lane == 0) a.lse[(static_cast<int64_t>(b) * a.H + h) * a.N_q + iq] = lse_tot;
   }
 }

@@ -62,24 +62,42 @@ static_assert(2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsOther <= kFwdThreads * k
 constexpr float kTau = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D>
+template <int D, Elem E = Elem::kBf16>
 struct FwdCfg {
-  static constexpr int kChunks = D / 64;               // 64-column (128-byte) swizzle chunks per row
-  static constexpr int kTileBytes = 128 * D * 2;       // one 128-row bf16 tile
-  static constexpr int kChunkBytes = 128 * 128;        // one 128-row x 64-column chunk
-  static constexpr int kStages = (D == 128) ? 4 : 8;   // K/V ring slots
+  static constexpr int kBytes = (E == Elem::kE4M3) ? 1 : 2;    // bytes per element
+  static constexpr int kRowBytes = D * kBytes;
+  static constexpr int kChunks = kRowBytes / 128;              // 128-byte swizzle chunks per row
+  static constexpr int kChunkElems = 128 / kBytes;             // elements per chunk row
+  static constexpr int kTileBytes = 128 * kRowBytes;           // one 128-row tile
+  static constexpr int kChunkBytes = 128 * 128;                // one 128-row x 128-byte chunk
+  static constexpr int kStages = (131072 / kTileBytes) < 16 ? (131072 / kTileBytes) : 16;  // K/V ring slots
+  static constexpr int kSSteps = kRowBytes / 32;               // MMA K-steps of S = Q K^T (32 bytes each)
+  static constexpr int kPVSteps = kBN * kBytes / 32;           // MMA K-steps of O += P V
+  static constexpr int kKeysPerStep = 32 / kBytes;
+  static constexpr int kPCols = kBN * kBytes / 4;              // TMEM columns of one P row
   static constexpr uint32_t kOCol = 256;
   static constexpr uint32_t kTmemCols = 512;
+  static_assert(kChunks >= 1, "rows of at least 128 bytes");
 };
 
-template <int D>
+// Output element type: the input type for 16-bit inputs, bf16 for e4m3 inputs.
+template <Elem E>
+struct FwdOut {
+  using T = typename ElemOps<E>::T;
+};
+template <>
+struct FwdOut<Elem::kE4M3> {
+  using T = __nv_bfloat16;
+};
+
+template <int D, Elem E = Elem::kBf16>
 struct __align__(1024) FwdSmem {
-  uint8_t q[2][FwdCfg<D>::kTileBytes];
-  uint8_t kv[FwdCfg<D>::kStages][FwdCfg<D>::kTileBytes];
+  uint8_t q[2][FwdCfg<D, E>::kTileBytes];
+  uint8_t kv[FwdCfg<D, E>::kStages][FwdCfg<D, E>::kTileBytes];
   uint64_t q_full[2];
   uint64_t q_empty[2];
-  uint64_t kv_full[FwdCfg<D>::kStages];
-  uint64_t kv_empty[FwdCfg<D>::kStages];
+  uint64_t kv_full[FwdCfg<D, E>::kStages];
+  uint64_t kv_empty[FwdCfg<D, E>::kStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_done[2];
@@ -149,9 +167,10 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 
 // Probabilities of one 128-key score row: p = 2^(s * scale_log2 - m), packed to bf16
 // pairs in p[]; adds the fp32 sum to *l and the sum of the bf16-rounded values to *lr.
-template <bool EMU>
+template <bool EMU, Elem E = Elem::kBf16>
 __device__ __forceinline__ void softmax_row(const uint32_t (&s)[kBN], uint32_t (&p)[kBN / 2], float scale_log2,
                                             float m, float& l, float& lr) {
+  static_assert(E != Elem::kE4M3, "e4m3 rows use softmax_row_e4m3");
   const float2 sl2 = make_float2(scale_log2, scale_log2);
   const float2 nm2 = make_float2(-m, -m);
   float2 se[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -166,27 +185,54 @@ __device__ __forceinline__ void softmax_row(const uint32_t (&s)[kBN], uint32_t (
       e.x = ex2_approx(x.x);
       e.y = ex2_approx(x.y);
     }
-    p[c] = pack_bf16x2(e.x, e.y);
+    p[c] = ElemOps<E>::pack(e.x, e.y);
     se[c & 1] = fadd2(se[c & 1], e);
     // the bf16 weights the P.V product actually uses: O = O_acc / lr is an exact
-    // convex combination of value rows (the rounding of a dominant weight cancels)
-    sr[c & 1] = fadd2(sr[c & 1], make_float2(__uint_as_float(p[c] << 16), __uint_as_float(p[c] & 0xffff0000u)));
+    // convex combination of value rows (the rounding of a dominant weight cancels).
+    // fp16 rounds 8x finer, so there lr is the fp32 sum itself.
+    if constexpr (E == Elem::kBf16) sr[c & 1] = fadd2(sr[c & 1], ElemOps<E>::unpack(p[c]));
+  }
+  const float ls = (se[0].x + se[0].y) + (se[1].x + se[1].y);
+  l += ls;
+  if constexpr (E == Elem::kBf16)
+    lr += (sr[0].x + sr[0].y) + (sr[1].x + sr[1].y);
+  else
+    lr += ls;
+}
+
+// e4m3 probabilities of one 128-key score row, four per word (first key in the lowest
+// byte); l gets the fp32 sum, lr the sum of the e4m3-rounded values the P.V product uses.
+__device__ __forceinline__ void softmax_row_e4m3(const uint32_t (&s)[kBN], uint32_t (&p)[kBN / 4],
+                                                 float scale_log2, float m, float& l, float& lr) {
+  const float2 sl2 = make_float2(scale_log2, scale_log2);
+  const float2 nm2 = make_float2(-m, -m);
+  float2 se[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 sr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < kBN / 4; ++c) {
+    const float2 x0 = ffma2(make_float2(__uint_as_float(s[4 * c]), __uint_as_float(s[4 * c + 1])), sl2, nm2);
+    const float2 x1 = ffma2(make_float2(__uint_as_float(s[4 * c + 2]), __uint_as_float(s[4 * c + 3])), sl2, nm2);
+    const float2 e0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+    const float2 e1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+    p[c] = pack_e4m3x4(e0.x, e0.y, e1.x, e1.y);
+    se[c & 1] = fadd2(se[c & 1], fadd2(e0, e1));
+    sr[c & 1] = fadd2(sr[c & 1], e4m3x4_pair_sums(p[c]));
   }
   l += (se[0].x + se[0].y) + (se[1].x + se[1].y);
   lr += (sr[0].x + sr[0].y) + (sr[1].x + sr[1].y);
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, Elem E = Elem::kBf16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
+                  const __grid_constant__ CUtensorMap tm_v, typename FwdOut<E>::T* __restrict__ out,
                   float* __restrict__ lse, int B, int H, int H_kv, int N, int window, float scale_log2,
-                  int* status) {
-  using Cfg = FwdCfg<D>;
+                  float out_scale, int* status) {
+  using Cfg = FwdCfg<D, E>;
   constexpr int NS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
-  FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                  ~static_cast<uintptr_t>(1023));
+  FwdSmem<D, E>& sm = *reinterpret_cast<FwdSmem<D, E>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                        ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int nkb = (N + kBN - 1) / kBN;
@@ -247,8 +293,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (!ok) break;
           mbar_arrive_expect_tx(&sm.q_full[i], Cfg::kTileBytes);
           for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_4d(sm.q[i] + c * Cfg::kChunkBytes, &tm_q, &sm.q_full[i], c * 64, ti.h, (ti.qb0 + i) * kBM,
-                        ti.b);
+            tma_load_4d(sm.q[i] + c * Cfg::kChunkBytes, &tm_q, &sm.q_full[i], c * Cfg::kChunkElems, ti.h,
+                        (ti.qb0 + i) * kBM, ti.b);
           ++qcnt[i];
         }
         // K/V stream: the union of both blocks' ranges (block 1's range starts and ends later)
@@ -262,7 +308,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_arrive_expect_tx(&sm.kv_full[s], Cfg::kTileBytes);
             const CUtensorMap* m = kv ? &tm_v : &tm_k;
             for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_4d(sm.kv[s] + c * Cfg::kChunkBytes, m, &sm.kv_full[s], c * 64, hkv, j * kBN, ti.b);
+              tma_load_4d(sm.kv[s] + c * Cfg::kChunkBytes, m, &sm.kv_full[s], c * Cfg::kChunkElems, hkv, j * kBN,
+                          ti.b);
           }
         }
       }
@@ -278,8 +325,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const WaitCtx wc{&sm.abort_flag, status, 2};
-      constexpr uint32_t idesc_s = idesc_bf16(128, kBN, 0, 0);  // Q, K both K-major
-      constexpr uint32_t idesc_o = idesc_bf16(128, D, 0, 1);    // P from TMEM, V MN-major
+      constexpr uint32_t idesc_s = idesc_kind_f16(128, kBN, 0, 0, ElemOps<E>::kMmaType);  // Q, K K-major
+      constexpr uint32_t idesc_o = idesc_kind_f16(128, D, 0, 1, ElemOps<E>::kMmaType);    // P in TMEM, V MN-major
       const uint32_t q_addr[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
       const uint32_t kv_addr0 = smem_u32(sm.kv[0]);
       uint32_t it = 0, qcnt[2] = {0, 0}, pcnt[2] = {0, 0};
@@ -294,9 +341,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t tS = tbase + i * 128;
         const uint64_t dk = dk0 + static_cast<uint64_t>((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < Cfg::kSSteps; ++kk) {
           const uint32_t off = ((kk / 4) * Cfg::kChunkBytes + (kk % 4) * 32) >> 4;
-          umma_ss(tS, dq[i] + off, dk + off, idesc_s, kk > 0);
+          if constexpr (E == Elem::kE4M3)
+            umma_ss_f8(tS, dq[i] + off, dk + off, idesc_s, kk > 0);
+          else
+            umma_ss(tS, dq[i] + off, dk + off, idesc_s, kk > 0);
         }
       };
       auto issue_pv = [&](int i, int slot, uint32_t acc) {
@@ -304,8 +354,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t tP = tbase + i * 128;
         const uint64_t dv = dv0 + static_cast<uint64_t>((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_o, (kk > 0) || acc);
+        for (int kk = 0; kk < Cfg::kPVSteps; ++kk) {
+          if constexpr (E == Elem::kE4M3)
+            umma_ts_f8(tO, tP + kk * 8, dv + ((kk * Cfg::kKeysPerStep * 128) >> 4), idesc_o, (kk > 0) || acc);
+          else
+            umma_ts(tO, tP + kk * 8, dv + ((kk * Cfg::kKeysPerStep * 128) >> 4), idesc_o, (kk > 0) || acc);
+        }
       };
 
       for (int k = 0; ok; ++k) {
@@ -452,17 +506,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_wait_st();
           }
         }
-        uint32_t p[kBN / 2];
+        uint32_t p[Cfg::kPCols];
         // a row that has seen no visible key yet (window edge) keeps m = -inf; use 0 as its
         // reference so that 2^(-inf - m) stays 0 instead of NaN
         const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
         // masked tiles hold -inf scores: they stay on the MUFU path (2^-inf = 0 exactly)
-        if (masked)
-          softmax_row<false>(s, p, scale_log2, m_use, l, lr);
-        else
-          softmax_row<true>(s, p, scale_log2, m_use, l, lr);
-        tmem_st32(tS + 0, p);
-        tmem_st32(tS + 32, p + 32);
+        if constexpr (E == Elem::kE4M3) {
+          softmax_row_e4m3(s, p, scale_log2, m_use, l, lr);
+          tmem_st32(tS + 0, p);
+        } else {
+          if (masked)
+            softmax_row<false, E>(s, p, scale_log2, m_use, l, lr);
+          else
+            softmax_row<true, E>(s, p, scale_log2, m_use, l, lr);
+          tmem_st32(tS + 0, p);
+          tmem_st32(tS + 32, p + 32);
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sm.p_full[g]);
@@ -473,9 +532,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (!ok) break;
       ++ocnt;
       tc_fence_after();
-      const float inv_l = 1.0f / lr;
+      // e4m3 inputs: out_scale is V's dequantisation factor
+      const float inv_l = (E == Elem::kE4M3 ? out_scale : 1.0f) / lr;
       const bool live = row < N;
-      __nv_bfloat16* orow = out + ((static_cast<int64_t>(ti.b) * N + row) * H + ti.h) * D;
+      typename FwdOut<E>::T* orow = out + ((static_cast<int64_t>(ti.b) * N + row) * H + ti.h) * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
@@ -484,7 +544,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 16; ++x)
-          pk[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv_l, __uint_as_float(o[2 * x + 1]) * inv_l);
+          pk[x] = ElemOps<E == Elem::kE4M3 ? Elem::kBf16 : E>::pack(__uint_as_float(o[2 * x]) * inv_l,
+                                                                   __uint_as_float(o[2 * x + 1]) * inv_l);
         if (live) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll

@@ -9,6 +9,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #ifndef FA_WAIT_TIMEOUT_NS
@@ -216,11 +217,12 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulator.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
+// Instruction descriptor, kind::f16 with fp32 accumulator; A and B both of `type`
+// (1 = bf16, 0 = f16).
+__host__ __device__ constexpr uint32_t idesc_kind_f16(int M, int N, int a_mn_major, int b_mn_major, uint32_t type = 1) {
   return (1u << 4)                                   // D: f32
-         | (1u << 7)                                 // A: bf16
-         | (1u << 10)                                // B: bf16
+         | (type << 7)                               // A format
+         | (type << 10)                              // B format
          | (static_cast<uint32_t>(a_mn_major) << 15)  // A major
          | (static_cast<uint32_t>(b_mn_major) << 16)  // B major
          | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
@@ -234,6 +236,28 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t adesc, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// kind::f8f6f4 (8-bit A and B, K = 32 per instruction): D[tmem] (+)= A[smem] * B[smem]
+__device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// kind::f8f6f4: D[tmem] (+)= A[tmem] * B[smem]
+__device__ __forceinline__ void umma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -358,5 +382,93 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
+  float2 r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "cvt.f32.f16 %0, lo;\n\t"
+      "cvt.f32.f16 %1, hi;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "r"(u));
+  return r;
+}
+
+// Four floats to e4m3 (round to nearest, saturating), first value in the lowest byte: the
+// byte order of a K-major row in tensor memory.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
+// The four e4m3 values of a packed word back to float (exact: every e4m3 value is an fp16
+// value).  Returns (a + b, c + d) of the decoded values a, b, c, d in byte order.
+__device__ __forceinline__ float2 e4m3x4_pair_sums(uint32_t u) {
+  float2 r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t.reg .b32 h0, h1;\n\t.reg .b16 a, b, c, d;\n\t"
+      ".reg .f32 fa, fb, fc, fd;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h0, lo;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h1, hi;\n\t"
+      "mov.b32 {a, b}, h0;\n\t"
+      "mov.b32 {c, d}, h1;\n\t"
+      "cvt.f32.f16 fa, a;\n\t"
+      "cvt.f32.f16 fb, b;\n\t"
+      "cvt.f32.f16 fc, c;\n\t"
+      "cvt.f32.f16 fd, d;\n\t"
+      "add.f32 %0, fa, fb;\n\t"
+      "add.f32 %1, fc, fd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "r"(u));
+  return r;
+}
+
+// ---------------------------------------------------------------- element types
+// The input types.  The 16-bit ones go through tcgen05 kind::f16 (the instruction
+// descriptor's A/B format field: 0 = f16, 1 = bf16), e4m3 through kind::f8f6f4 (format 0 =
+// E4M3, K = 32 per instruction); all accumulate in fp32.  A 16-bit row of D elements is
+// 2D bytes, an e4m3 row D bytes; shared-memory tiles keep 128-byte swizzled rows either way.
+enum class Elem : int { kBf16 = 0, kF16 = 1, kE4M3 = 2 };
+
+template <Elem E>
+struct ElemOps;
+
+template <>
+struct ElemOps<Elem::kBf16> {
+  using T = __nv_bfloat16;
+  static constexpr uint32_t kMmaType = 1;
+  __device__ static __forceinline__ uint32_t pack(float lo, float hi) { return pack_bf16x2(lo, hi); }
+  __device__ static __forceinline__ float2 unpack(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+  }
+  __device__ static __forceinline__ T one(float x) { return __float2bfloat16_rn(x); }
+};
+
+template <>
+struct ElemOps<Elem::kE4M3> {
+  using T = uint8_t;  // e4m3 bytes; the forward writes O in bf16
+  static constexpr uint32_t kMmaType = 0;
+};
+
+template <>
+struct ElemOps<Elem::kF16> {
+  using T = __half;
+  static constexpr uint32_t kMmaType = 0;
+  __device__ static __forceinline__ uint32_t pack(float lo, float hi) { return pack_f16x2(lo, hi); }
+  __device__ static __forceinline__ float2 unpack(uint32_t u) { return unpack_f16x2(u); }
+  __device__ static __forceinline__ T one(float x) { return __float2half_rn(x); }
+};
 
 }  // namespace fa

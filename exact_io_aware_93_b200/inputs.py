@@ -13,9 +13,9 @@ Recipe (the same for every workload):
 * For the peaked workload, a seeded permutation picks floor(N/100) sequence
   positions (shared by all batches and heads) and the whole K vector at those
   positions is multiplied by 3 in fp32, before rounding.
-* Every tensor is then rounded to bfloat16 (round to nearest even); the same
-  bf16 values are handed to the GPU and, widened exactly to fp64, to the
-  oracle.
+* Every tensor is then rounded to bfloat16 (round to nearest even), or to
+  float16 where a test asks for fp16; the same 16-bit values are handed to the
+  GPU and, widened exactly to fp64, to the oracle.
 * Checked query rows: per (b, h) a seeded sample without replacement from
   [0, N), always including rows 0, 1 and N-1.
 """
@@ -39,6 +39,7 @@ class Workload:
     peaked: bool = False
     H_kv: int | None = None          # key/value heads (None: same as H)
     window: int = -1                 # causal sliding window (-1: none)
+    dtype: str = "bf16"              # element type of the inputs: "bf16", "f16" or "e4m3" (forward only)
     # forward rows checked per head (None = every row)
     rows_per_head: int | None = None
     # backward: heads checked in full, plus (extra_heads x extra_rows_per_head) sampled rows
@@ -50,6 +51,10 @@ class Workload:
     @property
     def scale(self) -> float:
         return 1.0 / float(self.d) ** 0.5
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return {"f16": torch.float16, "e4m3": torch.float8_e4m3fn}.get(self.dtype, torch.bfloat16)
 
 
 # The five workloads: shapes, seeds and checked-row counts.
@@ -85,6 +90,12 @@ EXTRA_WORKLOADS = {
         Workload("window4096_causal_fwdbwd_b1_h32_hkv8_n32768_d128", 1, 32, 32768, 128, True, 1102,
                  backward=True, H_kv=8, window=4096,
                  notes="grouped heads + causal sliding window of 4096 keys, forward + backward"),
+        Workload("f16_causal_fwdbwd_b2_h16_n8192_d128", 2, 16, 8192, 128, True, 1104,
+                 backward=True, dtype="f16", bwd_full_heads=1, bwd_extra_heads=2, bwd_extra_rows=256,
+                 notes="the forward + backward configuration with fp16 tensors"),
+        Workload("e4m3_causal_fwd_b2_h16_n8192_d128", 2, 16, 8192, 128, True, 1105,
+                 dtype="e4m3", rows_per_head=256,
+                 notes="fp8 e4m3 forward at the forward + backward configuration's shape"),
     ]
 }
 
@@ -123,9 +134,10 @@ DECODE_WORKLOADS = {
 
 
 def make_decode_inputs(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int, seed: int, *,
-                       lengths="mixed", tail_nan: bool = False) -> dict[str, torch.Tensor]:
-    """CPU tensors for decoding: ``q`` bf16 [B, N_q, H, d], ``k``/``v`` bf16 [B, N_kv, H_kv, d]
-    (the cache) and ``seqlens`` int32 [B].
+                       lengths="mixed", tail_nan: bool = False,
+                       dtype: torch.dtype = torch.bfloat16) -> dict[str, torch.Tensor]:
+    """CPU tensors for decoding: ``q`` [B, N_q, H, d], ``k``/``v`` [B, N_kv, H_kv, d] (the
+    cache), bf16 unless ``dtype`` says float16, and ``seqlens`` int32 [B].
 
     Recipe: a ``torch.Generator('cpu')`` seeded with ``seed`` draws fp32 standard normals
     for q, k, v in that order, rounded to bf16; then the lengths: ``"full"`` gives N_kv
@@ -136,9 +148,9 @@ def make_decode_inputs(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int, s
     gen = torch.Generator(device="cpu")
     gen.manual_seed(int(seed))
     out = {
-        "q": torch.randn((B, N_q, H, d), generator=gen, dtype=torch.float32).to(torch.bfloat16),
-        "k": torch.randn((B, N_kv, H_kv, d), generator=gen, dtype=torch.float32).to(torch.bfloat16),
-        "v": torch.randn((B, N_kv, H_kv, d), generator=gen, dtype=torch.float32).to(torch.bfloat16),
+        "q": torch.randn((B, N_q, H, d), generator=gen, dtype=torch.float32).to(dtype),
+        "k": torch.randn((B, N_kv, H_kv, d), generator=gen, dtype=torch.float32).to(dtype),
+        "v": torch.randn((B, N_kv, H_kv, d), generator=gen, dtype=torch.float32).to(dtype),
     }
     if isinstance(lengths, str):
         if lengths == "full":
@@ -170,9 +182,10 @@ def peaked_positions(N: int, gen: torch.Generator) -> torch.Tensor:
 
 
 def make_inputs(B: int, H: int, N: int, d: int, seed: int, *, with_do: bool = False,
-                peaked: bool = False, H_kv: int | None = None) -> dict[str, torch.Tensor]:
-    """CPU bf16 tensors ``q`` (and ``do``) of shape [B, N, H, d] and ``k, v`` of shape
-    [B, N, H_kv, d] (H_kv defaults to H)."""
+                peaked: bool = False, H_kv: int | None = None,
+                dtype: torch.dtype = torch.bfloat16) -> dict[str, torch.Tensor]:
+    """CPU tensors ``q`` (and ``do``) of shape [B, N, H, d] and ``k, v`` of shape
+    [B, N, H_kv, d] (H_kv defaults to H), bf16 unless ``dtype`` says float16."""
     gen = torch.Generator(device="cpu")
     gen.manual_seed(int(seed))
     hkv = H if H_kv is None else int(H_kv)
@@ -186,12 +199,40 @@ def make_inputs(B: int, H: int, N: int, d: int, seed: int, *, with_do: bool = Fa
         out["k"][:, pos] *= 3.0
         out["peaked_positions"] = pos
     for name in names:
-        out[name] = out[name].to(torch.bfloat16)
+        out[name] = out[name].to(dtype)
+    return out
+
+
+def quantize_e4m3(x: torch.Tensor) -> tuple[torch.Tensor, float]:
+    """Per-tensor e4m3 quantisation: descale = fp32(amax / 448), so the largest magnitude lands
+    at the top of the e4m3 range, and codes = e4m3(x / descale) (round to nearest even,
+    computed in fp32).  The values the codes stand for are codes * descale."""
+    amax = float(x.abs().max())
+    descale = float(torch.tensor(amax / 448.0 if amax > 0 else 1.0, dtype=torch.float32))
+    codes = (x.to(torch.float32) / torch.tensor(descale, dtype=torch.float32)).to(torch.float8_e4m3fn)
+    return codes, descale
+
+
+def make_inputs_e4m3(B: int, H: int, N: int, d: int, seed: int, *, H_kv: int | None = None) -> dict:
+    """fp8 inputs: the fp32 normals of ``make_inputs`` (same generator order) quantised per
+    tensor with ``quantize_e4m3``.  Returns codes ``q, k, v`` (torch.float8_e4m3fn) and their
+    factors ``q_descale, k_descale, v_descale`` (Python floats holding fp32 values)."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    hkv = H if H_kv is None else int(H_kv)
+    out = {}
+    for name in ("q", "k", "v"):
+        heads = hkv if name in ("k", "v") else H
+        out[name], out[name + "_descale"] = quantize_e4m3(
+            torch.randn((B, N, heads, d), generator=gen, dtype=torch.float32))
     return out
 
 
 def make_workload_inputs(w: Workload) -> dict[str, torch.Tensor]:
-    return make_inputs(w.B, w.H, w.N, w.d, w.seed, with_do=w.backward, peaked=w.peaked, H_kv=w.H_kv)
+    if w.dtype == "e4m3":
+        return make_inputs_e4m3(w.B, w.H, w.N, w.d, w.seed, H_kv=w.H_kv)
+    return make_inputs(w.B, w.H, w.N, w.d, w.seed, with_do=w.backward, peaked=w.peaked, H_kv=w.H_kv,
+                       dtype=w.torch_dtype)
 
 
 def sample_rows(N: int, count: int | None, seed: int) -> torch.Tensor:

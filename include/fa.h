@@ -56,7 +56,7 @@ typedef enum {
   FA_ERR_WORKSPACE = 7    /* workspace pointer NULL or smaller than the required size */
 } fa_status;
 
-/* Library ABI version (this header: 3). */
+/* Library ABI version (this header: 4). */
 int fa_abi_version(void);
 
 /*
@@ -72,8 +72,16 @@ int fa_abi_version(void);
  *   causal       : 0 or 1
  *   window       : -1 for none; >= 0 (causal only) limits query i to keys i - window .. i,
  *                  sliding-window attention (same page, "Sliding Window Attention").
+ *   dtype        : element type of every tensor except lse: FA_DTYPE_BF16 or FA_DTYPE_F16
+ *                  (fp16, the type of the pages' memory example: "What Is Flash Attention?",
+ *                  bestllmfor.com, the score-matrix size table).  Arithmetic is the same:
+ *                  16-bit products, fp32 accumulation and softmax statistics.
+ *                  FA_DTYPE_E4M3 (forward only, d = 128): q, k, v are fp8 e4m3 bytes, o is
+ *                  bf16; see fa_fwd_e4m3_scaled.
  * Tensors: q, o, dO, dq are [B, N, H, d]; k, v, dk, dv are [B, N, H_kv, d]; lse is [B, H, N].
  */
+typedef enum { FA_DTYPE_BF16 = 0, FA_DTYPE_F16 = 1, FA_DTYPE_E4M3 = 2 } fa_dtype;
+
 typedef struct fa_problem {
   int B;
   int H;
@@ -83,6 +91,7 @@ typedef struct fa_problem {
   float scale;
   int causal;
   int window;
+  int dtype;
 } fa_problem;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -100,11 +109,28 @@ const char* fa_status_string(int status);
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  float scale, int causal, void* stream);
 
-/* fa_fwd for a general problem (grouped-query heads, sliding window).  Errors as fa_fwd,
- * plus FA_ERR_INVALID_ARG for a NULL problem, H_kv not dividing H, window < -1, or a
- * window without causal masking. */
+/* fa_fwd for a general problem (grouped-query heads, sliding window, bf16 or fp16 tensors).
+ * Errors as fa_fwd, plus FA_ERR_INVALID_ARG for a NULL problem, H_kv not dividing H,
+ * window < -1, or a window without causal masking, and FA_ERR_UNSUPPORTED for an unknown
+ * dtype. */
 fa_status fa_fwd_ex(const fa_problem* problem, const void* q, const void* k, const void* v, void* o,
                     float* lse, void* stream);
+
+/*
+ * Forward pass with fp8 e4m3 inputs (FlashAttention-3's FP8 forward: "Flash Attention
+ * Explained", institutepm.com, section "Flash Attention 1, 2, and 3").  problem->dtype must
+ * be FA_DTYPE_E4M3 and problem->d 128.  q, k, v hold e4m3 codes (1 byte per element, same
+ * [B, N, H(_kv), d] layout); the values they stand for are code * descale, one positive
+ * finite factor per tensor.  o is bf16 [B, N, H, d], lse fp32 [B, H, N] as in fa_fwd.
+ * Q K^T is formed exactly from the codes on the tensor cores (fp32 accumulation) and scaled
+ * by scale * q_descale * k_descale; the softmax weights are rounded to e4m3 for the P.V
+ * product and normalised by the sum of the rounded weights, O is scaled by v_descale; the
+ * LSE uses the unrounded fp32 sum.  fa_fwd_ex with this dtype is this call with descales 1.
+ * Errors as fa_fwd_ex, plus FA_ERR_INVALID_ARG for a dtype other than FA_DTYPE_E4M3 or a
+ * descale that is not positive and finite.
+ */
+fa_status fa_fwd_e4m3_scaled(const fa_problem* problem, const void* q, const void* k, const void* v,
+                             float q_descale, float k_descale, float v_descale, void* o, float* lse, void* stream);
 
 /*
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ accumulator
@@ -136,7 +162,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * B, H, N, d: the accumulator and statistics are per query head). 0 for a NULL problem. */
 size_t fa_bwd_workspace_size_ex(const fa_problem* problem);
 
-/* fa_bwd for a general problem: k, v, dk, dv are [B, N, H_kv, d]; dK and dV of a shared
+/* fa_bwd for a general problem (all 16-bit tensors in the problem's dtype; FA_DTYPE_E4M3
+ * returns FA_ERR_UNSUPPORTED): k, v, dk, dv are [B, N, H_kv, d]; dK and dV of a shared
  * key/value head accumulate the contributions of all H / H_kv query heads that use it.
  * Errors as fa_bwd, plus those of fa_fwd_ex for the problem. */
 fa_status fa_bwd_ex(const fa_problem* problem, const void* q, const void* k, const void* v, const void* o,
@@ -186,6 +213,7 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
  *              the cached prefix it extends, and sees the cached keys at or before that
  *              position; 0: every query sees all len_b cached keys
  *   window   : -1, or >= 0 with causal = 1: a query at position t sees keys t - window .. t
+ *   dtype    : FA_DTYPE_BF16 or FA_DTYPE_F16, the type of q, the caches and o
  * Constraint: (H / H_kv) * N_q <= 128 (the rows one key/value head contributes to a
  * 128-row tile); larger groups return FA_ERR_UNSUPPORTED.
  */
@@ -199,6 +227,7 @@ typedef struct fa_decode_problem {
   float scale;
   int causal;
   int window;
+  int dtype;
 } fa_decode_problem;
 
 /*

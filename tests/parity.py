@@ -30,6 +30,15 @@ def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
     return np.exp2(np.floor(np.log2(ax)) - 8)
 
 
+def half_ulp(x: np.ndarray, dtype: torch.dtype) -> np.ndarray:
+    """Half the spacing of the output type's grid at |x|: bf16 (8 significant bits) or
+    fp16 (11 significant bits; subnormal spacing below 2^-14)."""
+    if dtype == torch.float16:
+        ax = np.maximum(np.abs(x), 2.0 ** -14)
+        return np.exp2(np.floor(np.log2(ax)) - 11)
+    return bf16_half_ulp(x)
+
+
 def _head(t: torch.Tensor, b: int, h: int) -> np.ndarray:
     return t[b, :, h, :].to(torch.float64).numpy()
 
@@ -99,7 +108,7 @@ def fwd_errors_gqa(inputs, o_gpu, lse_gpu, scale, causal, window=-1, rows_per_he
                                              window=window)
             o_g = o_gpu[b, rows, h, :].to(torch.float64).numpy()
             l_g = lse_gpu[b, h, rows].to(torch.float64).numpy()
-            worst_o = max(worst_o, float((np.abs(o_g - o_ref) - bf16_half_ulp(o_ref)).max()))
+            worst_o = max(worst_o, float((np.abs(o_g - o_ref) - half_ulp(o_ref, o_gpu.dtype)).max()))
             worst_l = max(worst_l, float((np.abs(l_g - lse_ref) / np.maximum(1.0, np.abs(lse_ref))).max()))
     return worst_o, worst_l
 
@@ -144,6 +153,7 @@ def decode_errors(inputs, o_gpu, lse_gpu, scale, causal, window=-1, heads=None):
     pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
     o_g = o_gpu.cpu().double().numpy()
     l_g = lse_gpu.cpu().double().numpy()
+    out_dtype = o_gpu.dtype
     worst_o, worst_l = 0.0, 0.0
     for b, h in pairs:
         og, orf = o_g[b, :, h], o_ref[b, :, h]
@@ -153,8 +163,54 @@ def decode_errors(inputs, o_gpu, lse_gpu, scale, causal, window=-1, heads=None):
         empty = np.isneginf(lrf)
         if not np.array_equal(np.isneginf(lg), empty):
             return float("inf"), float("inf")
-        worst_o = max(worst_o, float((np.abs(og - orf) - bf16_half_ulp(orf)).max()))
+        worst_o = max(worst_o, float((np.abs(og - orf) - half_ulp(orf, out_dtype)).max()))
         if (~empty).any():
             worst_l = max(worst_l, float((np.abs(lg[~empty] - lrf[~empty]) /
                                           np.maximum(1.0, np.abs(lrf[~empty]))).max()))
     return worst_o, worst_l
+
+
+def e4m3_values(inputs, name: str) -> np.ndarray:
+    """The fp64 values e4m3 codes stand for: code * descale (exact in fp64)."""
+    return inputs[name].to(torch.float64).numpy() * float(inputs[name + "_descale"])
+
+
+def fwd_errors_e4m3(inputs, o_gpu, lse_gpu, scale, causal, window=-1, rows_per_head=None, seed=0, heads=None):
+    """Forward check for e4m3 inputs against the oracle on the dequantised values.
+
+    The kernel rounds the softmax weights to e4m3 before the P.V product and normalises by
+    their sum.  With w the exact weights of a row, p_j = 2^(x_j - m) for the kernel's
+    reference maximum m (at most 8 below the row maximum, never above it) and e4m3 rounding
+    error |p~_j - p_j| <= max(2^-4 p_j, 2^-10) (half an ulp in the normal range, half the
+    subnormal spacing below 2^-6), the output obeys
+        |O~_c - O_c| <= sum_j E_j |v_jc - O_c| / (1 - sum_j E_j),
+        E_j = max(2^-4 w_j, 2^-10 w_max)   over the visible keys j,
+    the worst case over m (m at the row maximum makes the absolute term largest).  Returns
+    (largest excess of |O~ - O| over that bound plus half a bf16 ulp and an fp32 slack of
+    1e-5 max|v| -- at most 0 when the bound holds --, largest |O~ - O|, LSE error)."""
+    q, k, v = (e4m3_values(inputs, n) for n in ("q", "k", "v"))
+    B, N, H, _ = q.shape
+    group = H // k.shape[2]
+    o_gpu, lse_gpu = o_gpu.cpu(), lse_gpu.cpu()
+    heads = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    excess, worst, worst_l = -np.inf, 0.0, 0.0
+    for b, h in heads:
+        qh, kh, vh = q[b, :, h], k[b, :, h // group], v[b, :, h // group]
+        rows = sample_rows(N, rows_per_head, head_row_seed(seed, b, h)).numpy()
+        o_ref, lse_ref = oracle.fwd_rows(qh, kh, vh, scale, causal, rows, window=window)
+        o_g = o_gpu[b, rows, h, :].to(torch.float64).numpy()
+        l_g = lse_gpu[b, h, rows].to(torch.float64).numpy()
+        worst_l = max(worst_l, float((np.abs(l_g - lse_ref) / np.maximum(1.0, np.abs(lse_ref))).max()))
+        slack = 1e-5 * np.abs(vh).max()
+        for r, i in enumerate(rows):
+            w = oracle.prob_row(qh, kh, scale, causal, int(i), window=window)
+            j = np.arange(N)
+            vis = (j <= i) if causal else np.ones(N, bool)
+            if window >= 0:
+                vis &= j >= i - window
+            e = np.where(vis, np.maximum(2.0 ** -4 * w, 2.0 ** -10 * w.max()), 0.0)
+            bound = (e @ np.abs(vh - o_ref[r])) / (1.0 - e.sum())
+            err = np.abs(o_g[r] - o_ref[r])
+            worst = max(worst, float(err.max()))
+            excess = max(excess, float((err - bound - bf16_half_ulp(o_ref[r]) - slack).max()))
+    return excess, worst, worst_l

@@ -46,7 +46,7 @@ def test_status_strings(lib):
     assert lib.fa_status_string(0) == b"FA_OK"
     assert lib.fa_status_string(6) == b"FA_ERR_TIMEOUT"
     assert lib.fa_status_string(99) == b"FA_ERR_UNKNOWN"
-    assert lib.fa_abi_version() == 3
+    assert lib.fa_abi_version() == 4
 
 
 def _fwd(lib, q=0x10000, k=0x10000, v=0x10000, o=0x10000, lse=0x10000, B=1, H=1, N=16, d=64,
@@ -135,6 +135,8 @@ def test_ex_validation_codes(lib):
     assert fwd(window=-2) == 1
     assert fwd(window=5, causal=0) == 1
     assert fwd(d=96) == 2
+    assert fwd(dtype=3) == 2 and fwd(dtype=-1) == 2   # bf16 (0), fp16 (1), e4m3 (2)
+    assert fwd(dtype=2, d=64) == 2                      # e4m3 is built for d = 128 only
     p = FaProblem(2, 4, 1, 100, 128, 0.1, 1, 16)
     assert lib.fa_bwd_workspace_size_ex(ctypes.byref(p)) == 4 * 2 * 4 * (100 * 128 + 2 * 128)
 
@@ -162,6 +164,7 @@ def test_decode_validation_codes(lib):
     assert dec(scale=0.0) == 1 and dec(causal=2) == 1
     assert dec(window=-2) == 1 and dec(window=4, causal=0) == 1
     assert dec(d=96) == 2
+    assert dec(dtype=5) == 2
     assert dec(H=8, H_kv=1, N_q=17) == 2       # 8 heads x 17 positions > 128 rows
     assert dec(H=8, H_kv=1, N_q=16) != 2
     assert dec(q=P + 8) == 3
@@ -172,3 +175,23 @@ def test_decode_validation_codes(lib):
         assert dec() == 4                       # valid problem, no sm_100 device here
         p = FaDecodeProblem(2, 8, 2, 1, 1000, 128, 0.1, 1, -1)
         assert lib.fa_decode_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_e4m3_validation_codes(lib):
+    from exact_io_aware_93_b200.api import FaProblem
+    vp = ctypes.c_void_p
+    f = ctypes.c_float
+    lib.fa_fwd_e4m3_scaled.argtypes = [ctypes.POINTER(FaProblem), vp, vp, vp, f, f, f, vp, vp, vp]
+    lib.fa_fwd_e4m3_scaled.restype = ctypes.c_int
+    P = 0x10000
+
+    def call(dtype=2, d=128, qd=1.0, kd=1.0, vd=1.0):
+        p = FaProblem(1, 2, 2, 64, d, 0.1, 1, -1, dtype)
+        return lib.fa_fwd_e4m3_scaled(ctypes.byref(p), vp(P), vp(P), vp(P), qd, kd, vd, vp(P), vp(P), None)
+    assert lib.fa_fwd_e4m3_scaled(None, vp(P), vp(P), vp(P), 1.0, 1.0, 1.0, vp(P), vp(P), None) == 1
+    assert call(dtype=0) == 1                 # this entry point is for e4m3 codes only
+    assert call(d=64) == 2
+    assert call(qd=0.0) == 1 and call(vd=float("inf")) == 1 and call(kd=-1.0) == 1
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == 4                    # valid, no sm_100 device here
