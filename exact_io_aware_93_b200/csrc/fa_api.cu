@@ -27,7 +27,7 @@ struct DeviceInfo {
   int* status = nullptr;
   bool fwd_attr[3][2][2] = {};  // [element type][d==128][causal]
   bool bwd_attr[2][2][2] = {};
-  bool dec_attr[2][2] = {};     // [fp16][d==128]
+  bool dec_attr[2][2][3] = {};  // [fp16][d==128][row copies 1, 2, 4]
 };
 DeviceInfo g_dev[kMaxDevices];
 
@@ -239,11 +239,13 @@ struct DecLayout {
 };
 
 // Workspace regions: schedule (total, tiles per CTA, per-sequence prefix), then the
-// partial log-sum-exps [S, M, 2] and partial outputs [S, M, d] of S = grid + B*H_kv - 1
-// slots (slot = CTA index + pair index is unique along the flattened tile list).
+// partial log-sum-exps [S, M, 2] and partial outputs [S, M, d] of S = R * (grid + B*H_kv - 1)
+// slots (slot = (CTA index + pair index) * R + row copy is unique along the flattened
+// tile list).
 DecLayout dec_layout(const fa_decode_problem& p, int grid) {
   const size_t M = static_cast<size_t>(p.H / p.H_kv) * p.N_q;
-  const size_t slots = static_cast<size_t>(grid) + static_cast<size_t>(p.B) * p.H_kv - 1;
+  const size_t slots = (static_cast<size_t>(grid) + static_cast<size_t>(p.B) * p.H_kv - 1) *
+                       static_cast<size_t>(fa::dec_copies(static_cast<int>(M)));
   DecLayout L;
   L.meta = 0;
   L.part_lse = round256((2 + static_cast<size_t>(p.B)) * 4);
@@ -256,9 +258,10 @@ template <int D, fa::Elem E>
 fa_status launch_decode(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         const fa_decode_problem& p, const int* seqlens, void* o, float* lse, void* ws,
                         cudaStream_t stream) {
-  auto kern = fa::fa_decode_kernel<D, E>;
+  const int R = fa::dec_copies((p.H / p.H_kv) * p.N_q);
+  auto kern = R == 4 ? fa::fa_decode_kernel<D, E, 4> : (R == 2 ? fa::fa_decode_kernel<D, E, 2> : fa::fa_decode_kernel<D, E, 1>);
   const int smem = static_cast<int>(sizeof(fa::DecSmem<D>)) + 1024;
-  bool& attr = di.dec_attr[E == fa::Elem::kF16][D == 128];
+  bool& attr = di.dec_attr[E == fa::Elem::kF16][D == 128][R >> 1];
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
       cudaGetLastError();
@@ -283,6 +286,7 @@ fa_status launch_decode(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap
   a.N_kv = p.N_kv;
   a.window = p.window;
   a.causal = p.causal;
+  a.R = R;
   a.scale_log2 = p.scale * 1.4426950408889634f;
   kern<<<grid, fa::kDecThreads, smem, stream>>>(mq, mk, mv, a, di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;

@@ -15,9 +15,14 @@
 // falls into SEGMENTS, each inside one pair.
 //
 // Rows.  The G = H / H_kv query heads that share a key/value head and the N_q new
-// positions form the rows of one 128-row tile, r = i*G + g ("Flash Attention Explained",
+// positions form the rows r = i*G + g of a tile ("Flash Attention Explained",
 // institutepm.com, "Grouped Query Attention"): the tile's K/V stream is read once for
-// all of them.  Rows at or past G*N_q are padding and are never written out.
+// all of them.  With M = G*N_q <= 32 (or <= 64) rows, R = 4 (or 2) copies of them fill the
+// 128 lanes, copy c at lanes [c*128/R, (c+1)*128/R), and copy c takes keys
+// [c*128/R, (c+1)*128/R) of every tile: each softmax warp then handles 128/R keys per
+// tile instead of 128, and the copies are independent online softmaxes over disjoint key
+// subsets, merged like any other partial results.  Lanes past a copy's M rows are padding
+// and are never written out.
 //
 // Two key streams.  The even tiles of a segment go to stream 0 and the odd tiles to
 // stream 1, each with its own score buffer, accumulator and row state, so the tensor core
@@ -25,9 +30,9 @@
 // it runs the other stream's products.  Each stream runs the prefill kernel's online
 // softmax (running maximum with conditional rescale, fp32 sum l for the LSE, bf16-rounded
 // sum lr for O).  At the end of a segment each thread merges its row's two streams with
-// log-sum-exp weights and writes the result: the final bf16 O and LSE when the segment
-// is the whole pair, otherwise an fp32 partial (O normalised, plus the natural-log sums
-// of l and of lr) that fa_decode_merge_kernel combines.
+// log-sum-exp weights and writes the result: the final O and LSE when the segment is the
+// whole pair and R = 1, otherwise an fp32 partial per copy (O normalised, plus the
+// natural-log sums of l and of lr) that fa_decode_merge_kernel combines.
 //
 // Stale cache.  Keys at or past a sequence's length are masked.  The value rows of a
 // tile past the length are zeroed in shared memory before the P.V product: a zero
@@ -86,14 +91,18 @@ struct __align__(1024) DecSmem {
   int abort_flag;
 };
 
+// Row copies per tile for M real rows: 4 when M <= 32, 2 when M <= 64, else 1.
+__host__ __device__ constexpr int dec_copies(int M) { return M <= 32 ? 4 : (M <= 64 ? 2 : 1); }
+
 struct DecArgs {
   const int* seqlens;      // [B] cached length of each sequence, or null: all N_kv
   void* out;               // [B, N_q, H, D], bf16 or fp16
   float* lse;              // [B, H, N_q]
   int* meta;               // [2 + B]: total tiles, tiles per CTA, per-sequence tile prefix
-  float* part_lse;         // [slots, M, 2]: natural-log sums of l and of lr of a segment
-  float* part_o;           // [slots, M, D]: segment output, normalised by its lr
+  float* part_lse;         // [slots * R, M, 2]: natural-log sums of l and of lr of a segment
+  float* part_o;           // [slots * R, M, D]: segment output, normalised by its lr
   int B, H, H_kv, N_q, N_kv, window, causal;
+  int R;                   // row copies per tile (dec_copies of M)
   float scale_log2;
 };
 
@@ -196,7 +205,7 @@ struct DecWalk {
   }
 };
 
-template <int D, Elem E = Elem::kBf16>
+template <int D, Elem E = Elem::kBf16, int R = 1>
 __global__ void __launch_bounds__(kDecThreads, 1)
     fa_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const DecArgs a, int* status) {
@@ -209,8 +218,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = a.H / a.H_kv;
-  const int M = G * a.N_q;          // real rows of the tile (<= 128)
-  const int aw = (M + 31) >> 5;     // softmax warps holding real rows
+  const int M = G * a.N_q;          // real rows of the tile (<= 128 / R)
+  constexpr int kWarpsPerCopy = 4 / R;
+  constexpr int kCopyRows = 128 / R;   // lanes per copy == keys per copy in a tile
+  // softmax warps holding real rows: the first ceil(M / 32) warps of every copy
+  const int aw = ((M + 31) >> 5) * R;
 
   if (threadIdx.x == 0) {
     sm.abort_flag = 0;
@@ -259,9 +271,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         ok = mbar_wait(&sm.q_empty[qi], ((qc >> 1) & 1) ^ 1, wc);
         if (!ok) break;
         // the G heads x N_q positions of this key/value head: one box per 64-column chunk
-        mbar_arrive_expect_tx(&sm.q_full[qi], static_cast<uint32_t>(Cfg::kChunks * 128 * M));
-        for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_4d(sm.q[qi] + c * Cfg::kChunkBytes, &tm_q, &sm.q_full[qi], c * 64, s.kvh * G, 0, s.b);
+        // and row copy (copy c at row c * 128 / R; a multiple of 8 rows keeps the swizzle)
+        mbar_arrive_expect_tx(&sm.q_full[qi], static_cast<uint32_t>(R * Cfg::kChunks * 128 * M));
+        for (int cp = 0; cp < R; ++cp)
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_4d(sm.q[qi] + c * Cfg::kChunkBytes + cp * kCopyRows * 128, &tm_q, &sm.q_full[qi], c * 64,
+                        s.kvh * G, 0, s.b);
         ++qc;
         // K/V tiles in the order the MMA warp consumes them: K0, K1, then V_t, K_{t+2}
         auto load = [&](const CUtensorMap* m, int t) -> bool {
@@ -395,13 +410,19 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mbar_wait_drain(&sm.mma_drain, 0, status);
     }
     __syncwarp();
-  } else if (warp < aw) {
+  } else if (warp < 4 && (warp % kWarpsPerCopy) * 32 < M) {
     // ------------------------------------------------------------ softmax, both streams
-    const int r = threadIdx.x;  // tile row == TMEM lane
+    constexpr int NC = kCopyRows;                 // keys of a tile this warp handles
+    const int cp = warp / kWarpsPerCopy;          // row copy
+    const int col0 = cp * NC;                     // its first key column in the tile
+    const int rc = (warp % kWarpsPerCopy) * 32 + lane;  // row within the copy
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t tS0 = tbase + lane_off;                 // stream i: + i * 128
     const uint32_t tO0 = tbase + Cfg::kOCol + lane_off;    // stream i: + i * D
     const WaitCtx wc{&sm.abort_flag, status, 23};
+    uint32_t zero[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) zero[x] = 0u;
     DecWalk w(plan);
     DecSeg s;
     uint32_t scnt0 = 0, scnt1 = 0, ocnt0 = 0, ocnt1 = 0;
@@ -413,39 +434,37 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       float mx_ = -INFINITY, lx = 0.f, lrx = 0.f;
       for (int t = 0; t < s.n; ++t) {
         const int i = t & 1;
-        const int k0 = (s.kt0 + t) * kBN;
+        const int k0 = (s.kt0 + t) * kBN + col0;    // this copy's first key
         const uint32_t tS = tS0 + i * 128;
         const uint32_t tO = tO0 + i * D;
         ok = __all_sync(kFull, mbar_wait(&sm.s_full[i], (i ? scnt1 : scnt0) & 1, wc));
         if (!ok) break;
         if (i) ++scnt1; else ++scnt0;
         tc_fence_after();
-        uint32_t sv[kBN];
-        tmem_ld32(tS + 0, sv + 0);
-        tmem_ld32(tS + 32, sv + 32);
-        tmem_ld32(tS + 64, sv + 64);
-        tmem_ld32(tS + 96, sv + 96);
+        uint32_t sv[NC];
+#pragma unroll
+        for (int c = 0; c < NC; c += 32) tmem_ld32(tS + col0 + c, sv + c);
         tmem_wait_ld();
         // every real row sees the keys up to all_hi and from all_lo on
         const int all_hi = a.causal ? s.len - a.N_q : s.len - 1;
         const int all_lo = a.window >= 0 ? s.len - 1 - a.window : 0;
-        const bool masked = (k0 + kBN - 1 > all_hi) || (k0 < all_lo);
+        const bool masked = (k0 + NC - 1 > all_hi) || (k0 < all_lo);
         if (masked) {
           // this row's visible keys: [vis_lo, vis_hi]
-          const int qpos = s.len - a.N_q + r / G;
-          const int vis_hi = r >= M ? -1 : (a.causal ? qpos : s.len - 1);
+          const int qpos = s.len - a.N_q + rc / G;
+          const int vis_hi = rc >= M ? -1 : (a.causal ? qpos : s.len - 1);
           const int vis_lo = a.window >= 0 ? qpos - a.window : 0;
           const int lim = vis_hi - k0;
           const int first = vis_lo - k0;
 #pragma unroll
-          for (int c = 0; c < kBN; ++c)
+          for (int c = 0; c < NC; ++c)
             if (c > lim || c < first) sv[c] = __float_as_uint(-INFINITY);
         }
         float mx8[8];
 #pragma unroll
         for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(__uint_as_float(sv[x]), __uint_as_float(sv[x + 8]));
 #pragma unroll
-        for (int c = 16; c < kBN; c += 16)
+        for (int c = 16; c < NC; c += 16)
 #pragma unroll
           for (int x = 0; x < 8; ++x)
             mx8[x] = fmax3(mx8[x], __uint_as_float(sv[c + x]), __uint_as_float(sv[c + 8 + x]));
@@ -475,14 +494,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             tmem_wait_st();
           }
         }
-        uint32_t p[kBN / 2];
+        uint32_t p[NC / 2];
         const float m_use = mc == -INFINITY ? 0.f : mc;
         if (masked)
-          softmax_row<false, E>(sv, p, a.scale_log2, m_use, lc, lrc);
+          softmax_row<false, E, NC>(sv, p, a.scale_log2, m_use, lc, lrc);
         else
-          softmax_row<true, E>(sv, p, a.scale_log2, m_use, lc, lrc);
-        tmem_st32(tS + 0, p);
-        tmem_st32(tS + 32, p + 32);
+          softmax_row<true, E, NC>(sv, p, a.scale_log2, m_use, lc, lrc);
+        // P for all 128 keys of the tile: this copy's columns, zeros for the other copies'
+#pragma unroll
+        for (int x = 0; x < NC / 2; x += 16) tmem_st16(tS + col0 / 2 + x, p + x);
+        if constexpr (R > 1) {
+#pragma unroll
+          for (int c = 0; c < 64; c += 16)
+            if (c < col0 / 2 || c >= col0 / 2 + NC / 2) tmem_st16(tS + c, zero);
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sm.p_full[i]);
@@ -516,11 +541,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const float inv = lrsum > 0.f ? 1.0f / lrsum : 0.f;
       const float lse_l = lsum > 0.f ? (mm + lg2_approx(lsum)) * kLn2 : -INFINITY;
       const float lse_r = lrsum > 0.f ? (mm + lg2_approx(lrsum)) * kLn2 : -INFINITY;
-      const bool real = r < M;
-      const int iq = r / G;  // new position of this row
+      const bool real = rc < M;
+      const bool direct = R == 1 && s.whole;
+      const int iq = rc / G;  // new position of this row
       const int b = s.p / a.H_kv;
-      const int h = (s.p - b * a.H_kv) * G + (r - iq * G);
-      const int64_t slot = static_cast<int64_t>(blockIdx.x) + s.p;
+      const int h = (s.p - b * a.H_kv) * G + (rc - iq * G);
+      const int64_t slot = (static_cast<int64_t>(blockIdx.x) + s.p) * R + cp;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t o0[32], o1[32];
@@ -532,7 +558,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         for (int x = 0; x < 32; ++x)
           v[x] = (a0 * __uint_as_float(o0[x]) + (has1 ? a1 * __uint_as_float(o1[x]) : 0.f)) * inv;
         if (real) {
-          if (s.whole) {
+          if (direct) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<typename ElemOps<E>::T*>(a.out) +
                                                   ((static_cast<int64_t>(b) * a.N_q + iq) * a.H + h) * D + c);
 #pragma unroll
@@ -541,18 +567,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                                   ElemOps<E>::pack(v[8 * x + 4], v[8 * x + 5]),
                                   ElemOps<E>::pack(v[8 * x + 6], v[8 * x + 7]));
           } else {
-            float4* dst = reinterpret_cast<float4*>(a.part_o + (slot * M + r) * D + c);
+            float4* dst = reinterpret_cast<float4*>(a.part_o + (slot * M + rc) * D + c);
 #pragma unroll
             for (int x = 0; x < 8; ++x) dst[x] = make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
           }
         }
       }
       if (real) {
-        if (s.whole) {
+        if (direct) {
           a.lse[(static_cast<int64_t>(b) * a.H + h) * a.N_q + iq] = lse_l;
         } else {
-          a.part_lse[(slot * M + r) * 2 + 0] = lse_l;
-          a.part_lse[(slot * M + r) * 2 + 1] = lse_r;
+          a.part_lse[(slot * M + rc) * 2 + 0] = lse_l;
+          a.part_lse[(slot * M + rc) * 2 + 1] = lse_r;
         }
       }
       tc_fence_before();
@@ -567,7 +593,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 }
 
-// Combines the partial results of the pairs whose tiles were split across CTAs: per row,
+// Combines the partial results of the pairs whose tiles were split across CTAs or row
+// copies: per row,
 // LSE = log sum_s exp(lse_s) and O = sum_s exp(lr_s - LR) O_s with LR = log sum_s exp(lr_s),
 // the same convex combination one CTA would have formed.  Pairs that one CTA covered were
 // written by it; pairs with no key (empty cache) get O = 0, LSE = -inf.  One block of four
@@ -597,11 +624,14 @@ __global__ void __launch_bounds__(128) fa_decode_merge_kernel(const DecArgs a) {
   const int start = a.meta[2 + b] + kvh * q.T;
   const int cf = start / per;
   const int cl = (start + q.T - 1) / per;
-  if (cf == cl) return;
+  if (cf == cl && a.R == 1) return;
+  // partial results of this pair: slots (c + p) * R + copy for CTAs c in [cf, cl]
+  const int s0 = (cf + p) * a.R;
+  const int s1 = (cl + p) * a.R + a.R - 1;
   for (int r = warp; r < M; r += 4) {
     float mx_l = -INFINITY, mx_r = -INFINITY;
-    for (int c = cf + lane; c <= cl; c += 32) {
-      const int64_t idx = ((static_cast<int64_t>(c) + p) * M + r) * 2;
+    for (int c = s0 + lane; c <= s1; c += 32) {
+      const int64_t idx = (static_cast<int64_t>(c) * M + r) * 2;
       mx_l = fmaxf(mx_l, a.part_lse[idx]);
       mx_r = fmaxf(mx_r, a.part_lse[idx + 1]);
     }
@@ -612,8 +642,8 @@ __global__ void __launch_bounds__(128) fa_decode_merge_kernel(const DecArgs a) {
     }
     float s_l = 0.f, s_r = 0.f;
     if (mx_r != -INFINITY) {
-      for (int c = cf + lane; c <= cl; c += 32) {
-        const int64_t idx = ((static_cast<int64_t>(c) + p) * M + r) * 2;
+      for (int c = s0 + lane; c <= s1; c += 32) {
+        const int64_t idx = (static_cast<int64_t>(c) * M + r) * 2;
         s_l += expf(a.part_lse[idx] - mx_l);
         s_r += expf(a.part_lse[idx + 1] - mx_r);
       }
@@ -629,8 +659,8 @@ __global__ void __launch_bounds__(128) fa_decode_merge_kernel(const DecArgs a) {
 #pragma unroll
     for (int j = 0; j < D / 32; ++j) acc[j] = 0.f;
     if (lr_tot != -INFINITY) {
-      for (int c = cf; c <= cl; ++c) {
-        const int64_t row = (static_cast<int64_t>(c) + p) * M + r;
+      for (int c = s0; c <= s1; ++c) {
+        const int64_t row = static_cast<int64_t>(c) * M + r;
         const float lr_s = a.part_lse[row * 2 + 1];
         if (lr_s == -INFINITY) continue;
         const float wgt = expf(lr_s - lr_tot);

@@ -165,18 +165,20 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 #define FA_FWD_EMU_MASK 0x00u
 #endif
 
-// Probabilities of one 128-key score row: p = 2^(s * scale_log2 - m), packed to bf16
-// pairs in p[]; adds the fp32 sum to *l and the sum of the bf16-rounded values to *lr.
-template <bool EMU, Elem E = Elem::kBf16>
-__device__ __forceinline__ void softmax_row(const uint32_t (&s)[kBN], uint32_t (&p)[kBN / 2], float scale_log2,
+// Probabilities of one score row of NC keys (128 in the prefill kernel): p = 2^(s *
+// scale_log2 - m), packed to 16-bit pairs in p[]; adds the fp32 sum to *l and the sum of
+// the bf16-rounded values to *lr.
+template <bool EMU, Elem E = Elem::kBf16, int NC = kBN>
+__device__ __forceinline__ void softmax_row(const uint32_t (&s)[NC], uint32_t (&p)[NC / 2], float scale_log2,
                                             float m, float& l, float& lr) {
   static_assert(E != Elem::kE4M3, "e4m3 rows use softmax_row_e4m3");
+  static_assert(NC % 4 == 0, "pairs alternate between two accumulators");
   const float2 sl2 = make_float2(scale_log2, scale_log2);
   const float2 nm2 = make_float2(-m, -m);
   float2 se[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   float2 sr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int c = 0; c < kBN / 2; ++c) {
+  for (int c = 0; c < NC / 2; ++c) {
     const float2 x = ffma2(make_float2(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sl2, nm2);
     float2 e;
     if (EMU && ((FA_FWD_EMU_MASK >> (c & 7)) & 1u)) {
