@@ -27,7 +27,7 @@ struct DeviceInfo {
   int* status = nullptr;
   bool fwd_attr[3][2][2] = {};  // [element type][d==128][causal]
   bool bwd_attr[2][2][2] = {};
-  bool dec_attr[2][2][3] = {};  // [fp16][d==128][row copies 1, 2, 4]
+  bool dec_attr[2][2][4] = {};  // [fp16][d==128][M = 128; M = 64 with 1, 2, 4 row copies]
 };
 DeviceInfo g_dev[kMaxDevices];
 
@@ -258,10 +258,14 @@ template <int D, fa::Elem E>
 fa_status launch_decode(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         const fa_decode_problem& p, const int* seqlens, void* o, float* lse, void* ws,
                         cudaStream_t stream) {
-  const int R = fa::dec_copies((p.H / p.H_kv) * p.N_q);
-  auto kern = R == 4 ? fa::fa_decode_kernel<D, E, 4> : (R == 2 ? fa::fa_decode_kernel<D, E, 2> : fa::fa_decode_kernel<D, E, 1>);
+  const int M = (p.H / p.H_kv) * p.N_q;
+  const int R = fa::dec_copies(M);
+  const bool m64 = fa::dec_mma_rows(M) == 64;
+  auto kern = !m64 ? fa::fa_decode_kernel<D, E, 1, 128>
+                   : (R == 4 ? fa::fa_decode_kernel<D, E, 4, 64>
+                             : (R == 2 ? fa::fa_decode_kernel<D, E, 2, 64> : fa::fa_decode_kernel<D, E, 1, 64>));
   const int smem = static_cast<int>(sizeof(fa::DecSmem<D>)) + 1024;
-  bool& attr = di.dec_attr[E == fa::Elem::kF16][D == 128][R >> 1];
+  bool& attr = di.dec_attr[E == fa::Elem::kF16][D == 128][m64 ? 1 + (R >> 1) : 0];
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
       cudaGetLastError();

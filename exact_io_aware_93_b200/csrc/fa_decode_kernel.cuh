@@ -17,11 +17,13 @@
 // Rows.  The G = H / H_kv query heads that share a key/value head and the N_q new
 // positions form the rows r = i*G + g of a tile ("Flash Attention Explained",
 // institutepm.com, "Grouped Query Attention"): the tile's K/V stream is read once for
-// all of them.  With M = G*N_q <= 32 (or <= 64) rows, R = 4 (or 2) copies of them fill the
-// 128 lanes, copy c at lanes [c*128/R, (c+1)*128/R), and copy c takes keys
-// [c*128/R, (c+1)*128/R) of every tile: each softmax warp then handles 128/R keys per
-// tile instead of 128, and the copies are independent online softmaxes over disjoint key
-// subsets, merged like any other partial results.  Lanes past a copy's M rows are padding
+// all of them.  Up to 64 rows use M = 64 MMAs, whose accumulators occupy lanes 0-15 of
+// each 32-lane quarter of tensor memory (half the tensor work of M = 128, which only
+// larger groups use).  The rows are copied to fill the tile: with M = G*N_q <= 16 (or
+// <= 32) rows, R = 4 (or 2) copies, copy c in quarters [c*4/R, (c+1)*4/R); copy c takes
+// keys [c*128/R, (c+1)*128/R) of every tile, so each softmax warp handles 128/R keys per
+// tile instead of 128.  The copies are independent online softmaxes over disjoint key
+// subsets, merged like any other partial results.  Lanes past a copy's rows are padding
 // and are never written out.
 //
 // Two key streams.  The even tiles of a segment go to stream 0 and the odd tiles to
@@ -39,7 +41,7 @@
 // weight times a stale NaN would still be NaN.
 //
 // Warp roles (192 threads, so up to 255 registers each): warps 0-3 softmax of both streams
-// (one thread per tile row; only the ceil(G*N_q / 32) warps holding real rows take part),
+// (one thread per tile row; only the warps holding real rows take part),
 // warp 4 TMA producer, warp 5 MMA issuer.  The cache stream, not the softmax, bounds the
 // kernel: at full HBM bandwidth one SM has ~2800 cycles per 128-key tile.
 //
@@ -91,8 +93,10 @@ struct __align__(1024) DecSmem {
   int abort_flag;
 };
 
-// Row copies per tile for M real rows: 4 when M <= 32, 2 when M <= 64, else 1.
-__host__ __device__ constexpr int dec_copies(int M) { return M <= 32 ? 4 : (M <= 64 ? 2 : 1); }
+// MMA rows for M real rows (64 when they fit, else 128) and row copies per tile: 4 when
+// M <= 16, 2 when M <= 32, else 1.
+__host__ __device__ constexpr int dec_mma_rows(int M) { return M <= 64 ? 64 : 128; }
+__host__ __device__ constexpr int dec_copies(int M) { return M <= 16 ? 4 : (M <= 32 ? 2 : 1); }
 
 struct DecArgs {
   const int* seqlens;      // [B] cached length of each sequence, or null: all N_kv
@@ -205,7 +209,7 @@ struct DecWalk {
   }
 };
 
-template <int D, Elem E = Elem::kBf16, int R = 1>
+template <int D, Elem E = Elem::kBf16, int R = 1, int kM = 128>
 __global__ void __launch_bounds__(kDecThreads, 1)
     fa_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const DecArgs a, int* status) {
@@ -218,11 +222,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = a.H / a.H_kv;
-  const int M = G * a.N_q;          // real rows of the tile (<= 128 / R)
+  const int M = G * a.N_q;              // real rows of a copy (<= kM / R)
+  static_assert(kM == 64 || kM == 128, "tcgen05 M of one CTA");
+  constexpr int kQuarterRows = kM / 4;     // accumulator lanes used per 32-lane quarter
   constexpr int kWarpsPerCopy = 4 / R;
-  constexpr int kCopyRows = 128 / R;   // lanes per copy == keys per copy in a tile
-  // softmax warps holding real rows: the first ceil(M / 32) warps of every copy
-  const int aw = ((M + 31) >> 5) * R;
+  constexpr int kCopyRows = kM / R;        // tile rows per copy
+  constexpr int kCopyKeys = 128 / R;       // keys per copy in a tile
+  // softmax warps holding real rows: the first ceil(M / kQuarterRows) warps of every copy
+  const int aw = ((M + kQuarterRows - 1) / kQuarterRows) * R;
 
   if (threadIdx.x == 0) {
     sm.abort_flag = 0;
@@ -304,8 +311,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // waits; lane 0 issues; the warp zeroes stale value rows)
     const WaitCtx wc{&sm.abort_flag, status, 22};
     const bool leader = lane == 0;
-    constexpr uint32_t idesc_s = idesc_kind_f16(128, kBN, 0, 0, ElemOps<E>::kMmaType);  // Q, K K-major
-    constexpr uint32_t idesc_o = idesc_kind_f16(128, D, 0, 1, ElemOps<E>::kMmaType);    // P in TMEM, V MN-major
+    constexpr uint32_t idesc_s = idesc_kind_f16(kM, kBN, 0, 0, ElemOps<E>::kMmaType);  // Q, K K-major
+    constexpr uint32_t idesc_o = idesc_kind_f16(kM, D, 0, 1, ElemOps<E>::kMmaType);    // P in TMEM, V MN-major
     const uint32_t kv_addr0 = smem_u32(sm.kv[0]);
     const uint64_t dq0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
     const uint64_t dq1 = sdesc_sw128(smem_u32(sm.q[1]), 16, 1024);
@@ -410,12 +417,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mbar_wait_drain(&sm.mma_drain, 0, status);
     }
     __syncwarp();
-  } else if (warp < 4 && (warp % kWarpsPerCopy) * 32 < M) {
+  } else if (warp < 4 && (warp % kWarpsPerCopy) * kQuarterRows < M) {
     // ------------------------------------------------------------ softmax, both streams
-    constexpr int NC = kCopyRows;                 // keys of a tile this warp handles
+    constexpr int NC = kCopyKeys;                 // keys of a tile this warp handles
     const int cp = warp / kWarpsPerCopy;          // row copy
     const int col0 = cp * NC;                     // its first key column in the tile
-    const int rc = (warp % kWarpsPerCopy) * 32 + lane;  // row within the copy
+    // row within the copy; with M = 64 lanes 16-31 of the quarter hold no accumulator rows
+    const int rc = lane < kQuarterRows ? (warp % kWarpsPerCopy) * kQuarterRows + lane : 1 << 20;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t tS0 = tbase + lane_off;                 // stream i: + i * 128
     const uint32_t tO0 = tbase + Cfg::kOCol + lane_off;    // stream i: + i * D
