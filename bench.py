@@ -341,6 +341,24 @@ def run_ours(args, w):
     bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in events["bwd"]) if events["bwd"] else None
     status = api.get_status()
 
+    # ---------------- the forward pass on its own (same inputs, back to back): the rate the
+    # forward target refers to, next to its rate inside the fwd + bwd step above
+    fwd_only = None
+    if with_bwd:
+        def fwd_step():
+            _step_fn(api, t, w, False)()
+        for _ in range(3):
+            fwd_step()
+        torch.cuda.synchronize()
+        fonly_steps = max(3, min(args.steps, 100))
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(fonly_steps):
+            fwd_step()
+        g1.record()
+        torch.cuda.synchronize()
+        fwd_only = {"ms": g0.elapsed_time(g1) / fonly_steps, "steps": fonly_steps}
+
     # ---------------- end-to-end through the public API: pinned host in, results back
     host = {n: inp[n].pin_memory() for n in names}
     out_host = {n: torch.empty(t[n].shape, dtype=t[n].dtype).pin_memory()
@@ -370,6 +388,8 @@ def run_ours(args, w):
     if world > 1:
         ms, e2e_ms, fwd_ms, bwd_ms = max_over_ranks([ms, e2e_ms, fwd_ms, bwd_ms or 0.0], dev)
         bwd_ms = bwd_ms if with_bwd else None
+        if fwd_only is not None:
+            fwd_only["ms"] = max_over_ranks([fwd_only["ms"]], dev)[0]
 
     ff = fwd_flops(w.B, w.H, w.N, w.d, w.causal, w.window)
     fb = bwd_flops(w.B, w.H, w.N, w.d, w.causal, w.window) if with_bwd else 0.0
@@ -405,6 +425,10 @@ def run_ours(args, w):
                            ("fa_fwd_e4m3_scaled (the e4m3 path is forward only)" if is8 else
                             "fa_fwd only (backward not built)")},
         "fwd_tflops": fwd_tf, "fwd_ms": fwd_ms, "bwd_tflops": bwd_tf, "bwd_ms": bwd_ms,
+        "fwd_alone": None if fwd_only is None else {
+            "tflops": ff / (fwd_only["ms"] * 1e-3) / 1e12, "ms": fwd_only["ms"], "steps": fwd_only["steps"],
+            "pct_of_peak": 100.0 * ff / (fwd_only["ms"] * 1e-3) / 1e12 / peak,
+            "note": "fa_fwd alone, back to back on the same inputs; fwd_tflops is its rate inside the step"},
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": in_bytes,
