@@ -407,11 +407,14 @@ def run_ours(args, w):
         dom = {"kernel": "fa_bwd (pre + main + post)", "achieved": bwd_tf, "ms": bwd_ms, "key": "fa_bwd"}
     else:
         dom = {"kernel": "fa_fwd_kernel", "achieved": fwd_tf, "ms": fwd_ms, "key": "fa_fwd_kernel"}
-    roofline = {"bound": "tensor", "achieved": dom["achieved"], "peak": peak, "unit": "TFLOP/s",
-                "frac": dom["achieved"] / peak, "traffic": measured_traffic(dom["key"], w.name),
+    # The dominant kernel is timed inside a long back-to-back step, which runs at the board's
+    # power cap (sw_power_cap in the clock record): its denominator is the sustained peak.
+    roofline = {"bound": "tensor", "achieved": dom["achieved"], "peak": peak_sus, "unit": "TFLOP/s",
+                "frac": dom["achieved"] / peak_sus, "traffic": measured_traffic(dom["key"], w.name),
                 "kernel": dom["kernel"],
-                "peak_kind": f"{peak_kind} bf16 burst (cuBLAS 8192^3)" if not is8 else f"{peak_kind} burst",
-                "frac_of_sustained": dom["achieved"] / peak_sus,
+                "peak_kind": (f"{peak_kind} bf16 sustained (cuBLAS 8192^3 back to back at the power cap)"
+                              if not is8 else f"{peak_kind} sustained"),
+                "burst_peak": peak, "frac_of_burst": dom["achieved"] / peak,
                 "fwd_alg_bytes": fwd_bytes(w.B, w.H, w.N, w.d)}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
@@ -428,8 +431,10 @@ def run_ours(args, w):
         "fwd_alone": None if fwd_only is None else {
             "tflops": ff / (fwd_only["ms"] * 1e-3) / 1e12, "ms": fwd_only["ms"], "steps": fwd_only["steps"],
             "pct_of_peak": 100.0 * ff / (fwd_only["ms"] * 1e-3) / 1e12 / peak,
-            "note": "fa_fwd alone, back to back on the same inputs; fwd_tflops is its rate inside the step"},
+            "note": "fa_fwd alone, back to back on the same inputs, a short burst: against the burst peak; "
+                    "fwd_tflops is its rate inside the step"},
         "pct_of_peak": 100.0 * value / world / peak,
+        "pct_of_sustained_peak": 100.0 * value / world / peak_sus,
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": d2h_bytes, "ms_per_step": e2e_ms, "steps": e2e_steps},
