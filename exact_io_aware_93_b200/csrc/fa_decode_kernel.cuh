@@ -667,14 +667,23 @@ __global__ void __launch_bounds__(128) fa_decode_merge_kernel(const DecArgs a) {
 #pragma unroll
     for (int j = 0; j < D / 32; ++j) acc[j] = 0.f;
     if (lr_tot != -INFINITY) {
-      for (int c = s0; c <= s1; ++c) {
-        const int64_t row = static_cast<int64_t>(c) * M + r;
-        const float lr_s = a.part_lse[row * 2 + 1];
-        if (lr_s == -INFINITY) continue;
-        const float wgt = expf(lr_s - lr_tot);
-        const float* po = a.part_o + row * D;
+      // 32 slots at a time: lane t computes the weight of slot base + t, then the warp sums
+      // the slots' rows with the weights broadcast, loads independent of each other
+      for (int base = s0; base <= s1; base += 32) {
+        const int c = base + lane;
+        float wl = 0.f;
+        if (c <= s1) {
+          const float lr_s = a.part_lse[(static_cast<int64_t>(c) * M + r) * 2 + 1];
+          wl = lr_s == -INFINITY ? 0.f : expf(lr_s - lr_tot);
+        }
+        const int cnt = min(32, s1 - base + 1);
+#pragma unroll 2
+        for (int t = 0; t < cnt; ++t) {
+          const float wgt = __shfl_sync(kFull, wl, t);
+          const float* po = a.part_o + (static_cast<int64_t>(base + t) * M + r) * D;
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) acc[j] += wgt * po[lane + 32 * j];
+          for (int j = 0; j < D / 32; ++j) acc[j] = fmaf(wgt, po[lane + 32 * j], acc[j]);
+        }
       }
     }
     const int iq = r / G, h = kvh * G + (r - iq * G);
