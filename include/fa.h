@@ -234,7 +234,8 @@ typedef struct fa_decode_problem {
  * Bytes of device workspace fa_decode needs on the CURRENT device (the split over its SMs
  * sets the number of partial results): 256-byte-aligned regions for the schedule
  * (4 * (2 + B) bytes), the partial log-sum-exps (8 * S * M) and the partial outputs
- * (4 * S * M * d), with S = SMs + B * H_kv - 1 and M = (H / H_kv) * N_q.
+ * (4 * S * M * d), with M = (H / H_kv) * N_q and S = R * (SMs + B * H_kv - 1), where
+ * R = 4 when M <= 16, 2 when M <= 32, else 1 (the copies of a head group's rows a tile holds).
  * Returns 0 for an invalid or unsupported problem or without an sm_100 device.
  */
 size_t fa_decode_workspace_size(const fa_decode_problem* problem);
