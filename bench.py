@@ -42,6 +42,7 @@ from exact_io_aware_93_b200.inputs import (DECODE_WORKLOADS, EXTRA_WORKLOADS, WO
 from exact_io_aware_93_b200.replicas import max_over_ranks, whole_job_tflops, world as _world  # noqa: E402
 
 METRIC = "attention fwd/bwd TFLOPS and % of B200 dense-bf16 peak, causal N=2K–128K"
+NOMINAL_BF16_TFLOPS = 2250.0   # datasheet dense bf16 per GPU (the 2:4-sparse figure halved)
 DECODE_METRIC = "attention decode: key/value cache bytes streamed per second (GB/s) and % of B200 HBM bandwidth"
 DEFAULT_WORKLOAD = "causal_fwdbwd_b2_h16_n8192_d128"
 L2_BYTES = 126 * 1024 * 1024
@@ -379,6 +380,11 @@ def run_ours(args, w):
     ms = e0.elapsed_time(e1) / args.steps
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in events["fwd"])
     bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in events["bwd"]) if events["bwd"] else None
+    # per-step times (start of the forward to the end of the step's last kernel)
+    ends = events["bwd"] if events["bwd"] else events["fwd"]
+    per_step = sorted(f[0].elapsed_time(e[1]) for f, e in zip(events["fwd"], ends))
+    pct = lambda q: per_step[min(len(per_step) - 1, int(q * len(per_step)))]
+    step_dist = {"p10_ms": pct(0.10), "median_ms": pct(0.50), "p90_ms": pct(0.90)}
     status = api.get_status()
 
     # ---------------- the forward pass on its own (same inputs, back to back): the rate the
@@ -467,6 +473,8 @@ def run_ours(args, w):
                     "fwd_tflops is its rate inside the step"},
         "pct_of_peak": 100.0 * value / world / peak,
         "pct_of_sustained_peak": 100.0 * value / world / peak_sus,
+        "pct_of_nominal_peak": 100.0 * value / world / (NOMINAL_BF16_TFLOPS * (2 if is8 else 1)),
+        "step_ms_distribution": step_dist,
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": d2h_bytes, "ms_per_step": e2e_ms, "steps": e2e_steps,
@@ -482,6 +490,7 @@ def run_ours(args, w):
         cflops, cdt = cpu_sample(w, heads, threads, backward=with_bwd)
         line["cpu_baseline"] = {
             "value": cflops / cdt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "extrapolated_full_step_s": step_flops / (cflops / cdt),
             "sample": f"{heads} full heads of {w.name} (forward" + (" + backward" if with_bwd else "")
                       + f", fp64{'; bf16-drawn inputs, the oracle costs the same for any input type' if is8 else ''}),"
                       f" {cdt:.1f} s"}
