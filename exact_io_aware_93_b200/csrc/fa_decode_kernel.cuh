@@ -504,10 +504,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
         uint32_t p[NC / 2];
         const float m_use = mc == -INFINITY ? 0.f : mc;
-        if (masked)
-          softmax_row<false, E, NC>(sv, p, a.scale_log2, m_use, lc, lrc);
-        else
-          softmax_row<true, E, NC>(sv, p, a.scale_log2, m_use, lc, lrc);
+        softmax_row<E, NC>(sv, p, a.scale_log2, m_use, lc, lrc);
         // P for all 128 keys of the tile: this copy's columns, zeros for the other copies'
 #pragma unroll
         for (int x = 0; x < NC / 2; x += 16) tmem_st16(tS + col0 / 2 + x, p + x);

@@ -159,16 +159,10 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   return true;
 }
 
-// Which of the 64 column pairs of an unmasked score row take the FMA-pipe exp2
-// (bit c % 8 of the mask): the MUFU unit alone cannot keep pace with the tensor core.
-#ifndef FA_FWD_EMU_MASK
-#define FA_FWD_EMU_MASK 0x00u
-#endif
-
 // Probabilities of one score row of NC keys (128 in the prefill kernel): p = 2^(s *
 // scale_log2 - m), packed to 16-bit pairs in p[]; adds the fp32 sum to *l and the sum of
 // the bf16-rounded values to *lr.
-template <bool EMU, Elem E = Elem::kBf16, int NC = kBN>
+template <Elem E = Elem::kBf16, int NC = kBN>
 __device__ __forceinline__ void softmax_row(const uint32_t (&s)[NC], uint32_t (&p)[NC / 2], float scale_log2,
                                             float m, float& l, float& lr) {
   static_assert(E != Elem::kE4M3, "e4m3 rows use softmax_row_e4m3");
@@ -180,13 +174,7 @@ __device__ __forceinline__ void softmax_row(const uint32_t (&s)[NC], uint32_t (&
 #pragma unroll
   for (int c = 0; c < NC / 2; ++c) {
     const float2 x = ffma2(make_float2(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sl2, nm2);
-    float2 e;
-    if (EMU && ((FA_FWD_EMU_MASK >> (c & 7)) & 1u)) {
-      e = exp2_poly2(x);
-    } else {
-      e.x = ex2_approx(x.x);
-      e.y = ex2_approx(x.y);
-    }
+    const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
     p[c] = ElemOps<E>::pack(e.x, e.y);
     se[c & 1] = fadd2(se[c & 1], e);
     // the bf16 weights the P.V product actually uses: O = O_acc / lr is an exact
@@ -512,15 +500,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // a row that has seen no visible key yet (window edge) keeps m = -inf; use 0 as its
         // reference so that 2^(-inf - m) stays 0 instead of NaN
         const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-        // masked tiles hold -inf scores: they stay on the MUFU path (2^-inf = 0 exactly)
+        // masked scores are -inf, and ex2 of -inf is exactly 0
         if constexpr (E == Elem::kE4M3) {
           softmax_row_e4m3(s, p, scale_log2, m_use, l, lr);
           tmem_st32(tS + 0, p);
         } else {
-          if (masked)
-            softmax_row<false, E>(s, p, scale_log2, m_use, l, lr);
-          else
-            softmax_row<true, E>(s, p, scale_log2, m_use, l, lr);
+          softmax_row<E>(s, p, scale_log2, m_use, l, lr);
           tmem_st32(tS + 0, p);
           tmem_st32(tS + 32, p + 32);
         }

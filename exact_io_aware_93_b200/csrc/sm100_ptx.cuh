@@ -353,29 +353,6 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   return r;
 }
 
-// 2^x for two lanes on the FMA pipe (no MUFU).  x = n + f with n = rint(x) and
-// f in [-1/2, 1/2]; 2^f is a cubic whose coefficients were fitted here for minimum
-// relative error on that interval (max relative error 7.5e-5, far below the bf16
-// spacing the result is rounded to); 2^n is applied by adding n to the exponent
-// field.  Adding 1.5 * 2^23 rounds x to an integer held in the low mantissa bits,
-// and (bits(t) << 23) leaves exactly n << 23.  x is clamped to >= -126 so that the
-// exponent cannot wrap; callers only pass finite x <= 2^22.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 magic = make_float2(12582912.0f, 12582912.0f);
-  const float2 t = fadd2(x, magic);
-  const float2 n = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = fadd2(x, make_float2(-n.x, -n.y));
-  float2 q = ffma2(make_float2(0.055171482f, 0.055171482f), f, make_float2(0.24261090f, 0.24261090f));
-  q = ffma2(q, f, make_float2(0.69326097f, 0.69326097f));
-  q = ffma2(q, f, make_float2(0.99992812f, 0.99992812f));
-  float2 r;
-  r.x = __int_as_float(__float_as_int(t.x) * (1 << 23) + __float_as_int(q.x));
-  r.y = __int_as_float(__float_as_int(t.y) * (1 << 23) + __float_as_int(q.y));
-  return r;
-}
-
 // Two fp32 -> bf16x2 (round to nearest even); lo goes to the low 16 bits.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
