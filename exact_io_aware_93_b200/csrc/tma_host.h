@@ -71,18 +71,4 @@ inline bool make_decode_q_map(CUtensorMap* map, const void* base, int B, int N_q
   return r == CUDA_SUCCESS;
 }
 
-// A row-major [rows, cols] bf16 matrix as a 2-D map with boxes of box_rows x 64 columns (128-byte swizzle).
-inline bool make_2d_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
-  EncodeTiledFn enc = encode_tiled_fn();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 }  // namespace fa
