@@ -428,19 +428,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* lse2 = sm.lse2[st] + 64 * g;
       const float* dd = sm.dd[st] + 64 * g;
       // bf16 P^T of this key row for the warpgroup's 64 queries, packed in pairs; dS uses the
-      // same rounded values that enter dV = P^T dO
-      uint32_t pk_all[32];
+      // same rounded values that enter dV = P^T dO.  The two chunks share one copy of the
+      // loop body (the kernel's code must fit the SM's instruction cache next to the other
+      // roles' loops): each chunk's words land in p_hi and the previous chunk's move to p_lo,
+      // so no register array is indexed by the loop counter.
+      uint32_t p_lo[16], p_hi[16];
 #pragma unroll
+      for (int x = 0; x < 16; ++x) p_hi[x] = 0u;
+#pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
         tmem_ld32(tS + c * 32, sv);
         tmem_wait_ld();
-        uint32_t* pk = pk_all + 16 * c;
+        uint32_t pk[16];
         if (masked)
           bwd_p_chunk<true, E>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, qhi, pk);
         else
           bwd_p_chunk<false, E>(sv, lse2 + c * 32, sl2, c * 32, key_ok, qlim, qhi, pk);
         tmem_st16(tS + c * 16, pk);  // columns already read
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          p_lo[x] = p_hi[x];
+          p_hi[x] = pk[x];
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -448,8 +458,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.dp_full, idx & 1, wc));
       if (!ok) break;
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {  // p_lo holds this chunk's P^T words
         uint32_t dpv[32];
         tmem_ld32(tDP + c * 32, dpv);
         tmem_wait_ld();
@@ -459,9 +469,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int y = 0; y < 8; ++y) d4s[y] = reinterpret_cast<const float4*>(dd + c * 32)[y];
 #pragma unroll
         for (int x = 0; x < 32; x += 4) {
-          const int ql = c * 32 + x;
           const float4 d4 = d4s[x / 4];
-          const uint32_t pa = pk_all[ql / 2], pb = pk_all[ql / 2 + 1];
+          const uint32_t pa = p_lo[x / 2], pb = p_lo[x / 2 + 1];
           const float2 a = fmul2(ElemOps<E>::unpack(pa),
                                  fadd2(make_float2(__uint_as_float(dpv[x]), __uint_as_float(dpv[x + 1])),
                                        make_float2(-d4.x, -d4.y)));
@@ -479,6 +488,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           *reinterpret_cast<uint4*>(ds_row + u * 16) =
               make_uint4(dsk[4 * y], dsk[4 * y + 1], dsk[4 * y + 2], dsk[4 * y + 3]);
         }
+#pragma unroll
+        for (int x = 0; x < 16; ++x) p_lo[x] = p_hi[x];
       }
       fence_proxy_async_smem();
       tc_fence_before();
