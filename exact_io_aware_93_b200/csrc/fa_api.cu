@@ -427,7 +427,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  // the same size limits as fa_bwd, so that the product below cannot wrap around
+  if (check_common(B, H, N, d, 1.0f, 0) != FA_OK) return 0;
   return bwd_ws_bytes(B, H, N, d);
 }
 

@@ -136,7 +136,8 @@ fa_status fa_fwd_e4m3_scaled(const fa_problem* problem, const void* q, const voi
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ accumulator
  * [B, H, N, d], then the fp32 row sums D_i = sum_x dO_ix O_ix and the fp32 LSE_i * log2(e),
  * each [B*H, Npad] with Npad = N rounded up to a multiple of 128; in total
- * 4*B*H*(N*d + 2*Npad) bytes.  Returns 0 for invalid sizes (B, H, N < 1 or d not 64 / 128).
+ * 4*B*H*(N*d + 2*Npad) bytes.  Returns 0 for sizes fa_bwd rejects (B, H, N < 1, d not
+ * 64 / 128, or more elements than its index range allows).
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 

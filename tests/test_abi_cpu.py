@@ -92,6 +92,8 @@ def test_bwd_validation_codes(lib):
     ws = lib.fa_bwd_workspace_size(1, 1, 16, 64)
     assert ws == 4 * (16 * 64 + 2 * 128)
     assert lib.fa_bwd_workspace_size(1, 1, 16, 96) == 0
+    # beyond the index range fa_bwd accepts: 0, not a wrapped-around byte count
+    assert lib.fa_bwd_workspace_size(2**31 - 1, 2**31 - 1, 2**31 - 1, 128) == 0
 
     def call(p=0x10000, wsp=0x10000, wsb=ws, d=64, B=1, scale=0.125):
         return lib.fa_bwd(vp(p), vp(0x10000), vp(0x10000), vp(0x10000), vp(0x10000), vp(0x10000),
