@@ -129,6 +129,21 @@ def validate_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
         raise TypeError(f"q, k, v must share one dtype, got {q.dtype}, {k.dtype}, {v.dtype}")
 
 
+def check_buffer(name: str, t: torch.Tensor, shape, dtype: torch.dtype, device: torch.device) -> None:
+    """A caller-supplied output must match exactly: the library writes through its raw pointer,
+    so a smaller or misplaced buffer would be written out of bounds."""
+    if (not isinstance(t, torch.Tensor) or tuple(t.shape) != tuple(shape) or t.dtype != dtype
+            or t.device != device or not t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on {device}")
+
+
+def check_scratch(name: str, t: torch.Tensor, device: torch.device) -> None:
+    """A caller-supplied workspace: any dtype, contiguous, on the inputs' device (its byte size
+    is checked by the library)."""
+    if not isinstance(t, torch.Tensor) or t.device != device or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous tensor on {device}")
+
+
 def problem(q: torch.Tensor, k: torch.Tensor, causal: bool, scale: float | None,
             window: int | None) -> FaProblem:
     B, N, H, d = q.shape
@@ -145,11 +160,13 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     limits query i to keys i - window .. i."""
     validate_inputs(q, k, v)
     B, N, H, d = q.shape
+    out_dtype = torch.bfloat16 if q.dtype == torch.float8_e4m3fn else q.dtype
     if out is None:
-        out = torch.empty(q.shape, dtype=torch.bfloat16 if q.dtype == torch.float8_e4m3fn else q.dtype,
-                          device=q.device)
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    check_buffer("out", out, q.shape, out_dtype, q.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    check_buffer("lse", lse, (B, H, N), torch.float32, q.device)
     p = problem(q, k, causal, scale, window)
     st = lib().fa_fwd_ex(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                          lse.data_ptr(), _stream_ptr(q))
@@ -169,6 +186,8 @@ def fwd_e4m3(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_descale: float
     B, N, H, d = q.shape
     out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) if out is None else out
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    check_buffer("out", out, q.shape, torch.bfloat16, q.device)
+    check_buffer("lse", lse, (B, H, N), torch.float32, q.device)
     p = problem(q, k, causal, scale, window)
     st = lib().fa_fwd_e4m3_scaled(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                   float(q_descale), float(k_descale), float(v_descale), out.data_ptr(),
@@ -193,15 +212,18 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, do: 
         if t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous() or t.device != q.device:
             raise ValueError(f"{name} must be a contiguous tensor shaped like q, of q's dtype")
     B, N, H, d = q.shape
-    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
+    check_buffer("lse", lse, (B, H, N), torch.float32, q.device)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    check_buffer("dq", dq, q.shape, q.dtype, q.device)
+    check_buffer("dk", dk, k.shape, k.dtype, q.device)
+    check_buffer("dv", dv, v.shape, v.dtype, q.device)
     p = problem(q, k, causal, scale, window)
     need = int(lib().fa_bwd_workspace_size_ex(ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    check_scratch("workspace", workspace, q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     st = lib().fa_bwd_ex(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                          do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
@@ -245,15 +267,19 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
         raise ValueError(f"cache shapes {tuple(k_cache.shape)}, {tuple(v_cache.shape)} do not fit q {tuple(q.shape)}")
     if H % k_cache.shape[2] != 0:
         raise ValueError("key/value heads must divide the query heads")
-    if seqlens is not None and (seqlens.dtype != torch.int32 or seqlens.shape != (B,) or not seqlens.is_cuda
-                                or not seqlens.is_contiguous()):
-        raise ValueError("seqlens must be a contiguous int32 [B] CUDA tensor")
+    if not (k_cache.device == v_cache.device == q.device):
+        raise ValueError("q, k_cache and v_cache must be on the same device")
+    if seqlens is not None:
+        check_buffer("seqlens", seqlens, (B,), torch.int32, q.device)
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, H, n_q), dtype=torch.float32, device=q.device) if lse is None else lse
+    check_buffer("out", out, q.shape, q.dtype, q.device)
+    check_buffer("lse", lse, (B, H, n_q), torch.float32, q.device)
     p = decode_problem(q, k_cache, causal, scale, window)
     need = int(lib().fa_decode_workspace_size(ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    check_scratch("workspace", workspace, q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     st = lib().fa_decode(ctypes.byref(p), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
                          None if seqlens is None else seqlens.data_ptr(), out.data_ptr(), lse.data_ptr(),
