@@ -121,41 +121,75 @@ class ClockSampler:
         self.window = (t_begin, t_end)
 
     def stop(self):
+        """End sampling and return the statistics of the window given to mark()."""
+        self.close()
+        return self.stats(self.window)
+
+    def close(self):
+        """End sampling and read every sample; stats() then summarises any window."""
+        self.samples = []
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
-        import datetime
-        sm, smax, power, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 10:
-                    continue
-                try:
-                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                    clk, cmax = float(parts[2].split()[0]), float(parts[3].split()[0])
-                    pw = float(parts[4].split()[0])
-                except ValueError:
-                    continue
-                if self.window and not (self.window[0] - 0.05 <= ts <= self.window[1] + 0.05):
-                    continue
-                sm.append(clk)
-                smax.append(cmax)
-                power.append(pw)
-                for name, val in zip(names, parts[6:10]):
-                    if val.lower() == "active":
-                        reasons.add(name)
+            self.samples = parse_clock_samples(f)
         os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "power_w_max": max(power) if power else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+
+    def stats(self, window):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0, "power_cap_samples": 0,
+                    "reasons": ["nvidia-smi unavailable"]}
+        return clock_stats(self.samples, window)
+
+
+CLOCK_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+def parse_clock_samples(lines):
+    """Rows of the nvidia-smi query above as dicts (timestamp in seconds since the epoch)."""
+    import datetime
+    out = []
+    for line in lines:
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 10:
+            continue
+        try:
+            ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            clk, cmax = float(parts[2].split()[0]), float(parts[3].split()[0])
+            pw = float(parts[4].split()[0])
+        except ValueError:
+            continue
+        out.append({"ts": ts, "sm": clk, "sm_max": cmax, "power": pw,
+                    "reasons": [n for n, v in zip(CLOCK_REASONS, parts[6:10]) if v.lower() == "active"]})
+    return out
+
+
+def clock_stats(samples, window, slack_s: float = 0.05):
+    """Median SM clock, max clock, peak power and the throttle reasons of the samples taken
+    inside `window` (t_begin, t_end), with the number of samples that saw the power cap."""
+    sel = [x for x in samples if window is None or window[0] - slack_s <= x["ts"] <= window[1] + slack_s]
+    reasons = sorted({r for x in sel for r in x["reasons"]})
+    return {"sm_mhz": statistics.median(x["sm"] for x in sel) if sel else None,
+            "sm_max_mhz": max(x["sm_max"] for x in sel) if sel else None,
+            "power_w_max": max(x["power"] for x in sel) if sel else None,
+            "samples": len(sel),
+            "power_cap_samples": sum("sw_power_cap" in x["reasons"] for x in sel),
+            "reasons": reasons}
+
+
+def choose_peak(clk, burst: float, sustained: float):
+    """The tensor peak a timed region is compared with, chosen from that region's own clock
+    samples: the sustained (power-capped) cuBLAS figure when any in-region sample shows
+    sw_power_cap, else the burst figure.  Returns (peak, kind, rule)."""
+    n, capped = clk.get("samples", 0) or 0, clk.get("power_cap_samples", 0) or 0
+    if capped > 0:
+        return sustained, "sustained", f"sw_power_cap active in {capped} of {n} in-region clock samples"
+    return burst, "burst", f"sw_power_cap active in 0 of {n} in-region clock samples"
 
 
 def pipelined_e2e(sets, host_in, in_names, out_names, compute, nsteps):
@@ -321,18 +355,9 @@ def run_reference(args, w):
     return 0
 
 
-def run_ours(args, w):
-    world, rank, local = _dist_env()
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    from exact_io_aware_93_b200 import api
-    dev = torch.device("cuda", torch.cuda.current_device())
-    is8 = w.dtype == "e4m3"             # the e4m3 path is forward only
-    with_bwd = with_bwd_available() and not is8
-
+def _device_inputs(api, w, dev, with_bwd):
+    """Seeded inputs of workload w on the device plus its output buffers and workspace."""
+    is8 = w.dtype == "e4m3"
     if is8:
         inp = make_workload_inputs(w)
         names = ("q", "k", "v")
@@ -348,6 +373,100 @@ def run_ours(args, w):
     if with_bwd:
         t["dq"], t["dk"], t["dv"] = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
         t["ws"] = torch.empty(api.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    return inp, t, names
+
+
+def _timed_steps(api, t, w, with_bwd, nsteps, barrier=None):
+    """Time `nsteps` back-to-back steps with CUDA events on the launch stream.  Returns the
+    wall-clock window (for the clock samples), the mean step time and the mean forward and
+    backward times from per-step events."""
+    events = {"fwd": [], "bwd": []}
+    tstep = _step_fn(api, t, w, with_bwd, events)
+    if barrier is not None:
+        barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_begin = time.time()
+    e0.record()
+    for _ in range(nsteps):
+        tstep()
+    e1.record()
+    torch.cuda.synchronize()
+    t_end = time.time()
+    ms = e0.elapsed_time(e1) / nsteps
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in events["fwd"])
+    bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in events["bwd"]) if events["bwd"] else None
+    ends = events["bwd"] if events["bwd"] else events["fwd"]
+    per_step = sorted(f[0].elapsed_time(e[1]) for f, e in zip(events["fwd"], ends))
+    return {"window": (t_begin, t_end), "ms": ms, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "per_step": per_step}
+
+
+# The metric's sequence-length range: a fwd + bwd step of each causal configuration, each
+# timed for about PER_CONFIG_SECONDS with its own clock record.
+PER_CONFIG = ("causal_b4_h16_n2048_d128", "causal_fwdbwd_b2_h16_n8192_d128", "causal_b1_h32_n32768_d128",
+              "causal_peaked_b1_h8_n131072_d128")
+PER_CONFIG_SECONDS = 1.0
+
+
+def per_config_records(api, dev, clocks, burst, sustained, warmup):
+    """One record per PER_CONFIG workload: fwd_ms, bwd_ms, the step's TFLOP/s and the
+    fraction of the peak its own in-region clock samples select (choose_peak)."""
+    out = {}
+    for name in PER_CONFIG:
+        w = WORKLOADS[name]
+        inp, t, _ = _device_inputs(api, w, dev, True)
+        del inp
+        step = _step_fn(api, t, w, True)
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(warmup):
+            step()
+        g1.record()
+        torch.cuda.synchronize()
+        est_ms = g0.elapsed_time(g1) / warmup
+        nsteps = max(5, min(500, int(PER_CONFIG_SECONDS * 1e3 / max(est_ms, 1e-3))))
+        r = _timed_steps(api, t, w, True, nsteps)
+        out[name] = r
+        out[name]["steps"] = nsteps
+        out[name]["status"] = api.get_status()
+        del t
+        torch.cuda.empty_cache()
+    return out
+
+
+def _per_config_json(recs, clocks, burst, sustained):
+    js = {}
+    for name, r in recs.items():
+        w = WORKLOADS[name]
+        ff = fwd_flops(w.B, w.H, w.N, w.d, w.causal, w.window)
+        fb = bwd_flops(w.B, w.H, w.N, w.d, w.causal, w.window)
+        clk = clocks.stats(r["window"])
+        peak, kind, rule = choose_peak(clk, burst, sustained)
+        step_tf = (ff + fb) / (r["ms"] * 1e-3) / 1e12
+        fwd_tf = ff / (r["fwd_ms"] * 1e-3) / 1e12
+        bwd_tf = fb / (r["bwd_ms"] * 1e-3) / 1e12
+        js[name] = {"B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "peaked": w.peaked,
+                    "steps": r["steps"], "ms_per_step": r["ms"], "fwd_ms": r["fwd_ms"], "bwd_ms": r["bwd_ms"],
+                    "step_tflops": step_tf, "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+                    "peak": peak, "peak_kind": kind, "peak_rule": rule,
+                    "step_frac": step_tf / peak, "fwd_frac": fwd_tf / peak, "bwd_frac": bwd_tf / peak,
+                    "clocks": clk, "device_status": r["status"]}
+    return js
+
+
+def run_ours(args, w):
+    world, rank, local = _dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from exact_io_aware_93_b200 import api
+    dev = torch.device("cuda", torch.cuda.current_device())
+    is8 = w.dtype == "e4m3"             # the e4m3 path is forward only
+    with_bwd = with_bwd_available() and not is8
+    inp, t, names = _device_inputs(api, w, dev, with_bwd)
     in_bytes = sum(t[n].numel() * t[n].element_size() for n in names)
 
     step = _step_fn(api, t, w, with_bwd)
@@ -360,30 +479,14 @@ def run_ours(args, w):
         raise RuntimeError("device status word set during warm-up")
 
     # ---------------- device-timed region
-    events = {"fwd": [], "bwd": []}
-    tstep = _step_fn(api, t, w, with_bwd, events)
+    barrier = None
     if world > 1:
         import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_begin = time.time()
-    e0.record()
-    for _ in range(args.steps):
-        tstep()
-    e1.record()
-    torch.cuda.synchronize()
-    t_end = time.time()
+        barrier = dist.barrier
+    r = _timed_steps(api, t, w, with_bwd, args.steps, barrier)
     if world > 1:
         dist.barrier()
-    clocks.mark(t_begin, t_end)
-    clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in events["fwd"])
-    bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in events["bwd"]) if events["bwd"] else None
-    # per-step times (start of the forward to the end of the step's last kernel)
-    ends = events["bwd"] if events["bwd"] else events["fwd"]
-    per_step = sorted(f[0].elapsed_time(e[1]) for f, e in zip(events["fwd"], ends))
+    ms, fwd_ms, bwd_ms, per_step = r["ms"], r["fwd_ms"], r["bwd_ms"], r["per_step"]
     pct = lambda q: per_step[min(len(per_step) - 1, int(q * len(per_step)))]
     step_dist = {"p10_ms": pct(0.10), "median_ms": pct(0.50), "p90_ms": pct(0.90)}
     status = api.get_status()
@@ -395,7 +498,7 @@ def run_ours(args, w):
         def fwd_step():
             _step_fn(api, t, w, False)()
         # Timed as a burst, the way the burst peak it is compared with was measured: after a
-        # short idle pause rather than straight after the power-capped step loop above.
+        # short idle pause rather than straight after the step loop above.
         time.sleep(FWD_ALONE_PAUSE_S)
         for _ in range(3):
             fwd_step()
@@ -433,15 +536,25 @@ def run_ours(args, w):
         if fwd_only is not None:
             fwd_only["ms"] = max_over_ranks([fwd_only["ms"]], dev)[0]
 
+    peak, peak_sus, hbm, peak_kind = _peaks()
+    if is8:
+        # e4m3 contraction: the measured bf16 peak times the nominal dense e4m3 / bf16 ratio (2)
+        peak, peak_sus, peak_kind = 2 * peak, 2 * peak_sus, peak_kind + " bf16 x 2 (nominal e4m3/bf16 ratio);"
+
+    # ---------------- the metric's range: N = 2K, 8K, 32K, 128K, each with its own clocks
+    recs = None
+    if world == 1 and not args.no_per_config and w.name == DEFAULT_WORKLOAD and with_bwd:
+        del t2, sets
+        torch.cuda.empty_cache()
+        recs = per_config_records(api, dev, clocks, peak, peak_sus, 3)
+    clocks.close()
+    clk = clocks.stats(r["window"])
+
     ff = fwd_flops(w.B, w.H, w.N, w.d, w.causal, w.window)
     fb = bwd_flops(w.B, w.H, w.N, w.d, w.causal, w.window) if with_bwd else 0.0
     step_flops = ff + fb
     value = whole_job_tflops(world, step_flops, ms)
     e2e_value = whole_job_tflops(world, step_flops, e2e_ms)
-    peak, peak_sus, hbm, peak_kind = _peaks()
-    if is8:
-        # e4m3 contraction: the measured bf16 peak times the nominal dense e4m3 / bf16 ratio (2)
-        peak, peak_sus, peak_kind = 2 * peak, 2 * peak_sus, peak_kind + " bf16 x 2 (nominal e4m3/bf16 ratio);"
     fwd_tf = ff / (fwd_ms * 1e-3) / 1e12
     bwd_tf = fb / (bwd_ms * 1e-3) / 1e12 if with_bwd else None
     # dominant kernel: the one with the larger share of the step
@@ -449,14 +562,17 @@ def run_ours(args, w):
         dom = {"kernel": "fa_bwd (pre + main + post)", "achieved": bwd_tf, "ms": bwd_ms, "key": "fa_bwd"}
     else:
         dom = {"kernel": "fa_fwd_kernel", "achieved": fwd_tf, "ms": fwd_ms, "key": "fa_fwd_kernel"}
-    # The dominant kernel is timed inside a long back-to-back step, which runs at the board's
-    # power cap (sw_power_cap in the clock record): its denominator is the sustained peak.
-    roofline = {"bound": "tensor", "achieved": dom["achieved"], "peak": peak_sus, "unit": "TFLOP/s",
-                "frac": dom["achieved"] / peak_sus, "traffic": measured_traffic(dom["key"], w.name),
+    # The denominator follows the timed region's own clock samples: the sustained
+    # (power-capped) cuBLAS figure if any of them shows sw_power_cap, else the burst figure.
+    chosen, chosen_kind, rule = choose_peak(clk, peak, peak_sus)
+    roofline = {"bound": "tensor", "achieved": dom["achieved"], "peak": chosen, "unit": "TFLOP/s",
+                "frac": dom["achieved"] / chosen, "traffic": measured_traffic(dom["key"], w.name),
                 "kernel": dom["kernel"],
-                "peak_kind": (f"{peak_kind} bf16 sustained (cuBLAS 8192^3 back to back at the power cap)"
-                              if not is8 else f"{peak_kind} sustained"),
-                "burst_peak": peak, "frac_of_burst": dom["achieved"] / peak,
+                "peak_kind": f"{peak_kind} bf16 {chosen_kind} (cuBLAS bf16 8192^3"
+                             + (", back to back at the power cap)" if chosen_kind == "sustained" else ", burst)")
+                             + (" x 2 for e4m3" if is8 else ""),
+                "peak_rule": rule, "burst_peak": peak, "sustained_peak": peak_sus,
+                "frac_of_burst": dom["achieved"] / peak, "frac_of_sustained": dom["achieved"] / peak_sus,
                 "fwd_alg_bytes": fwd_bytes(w.B, w.H, w.N, w.d)}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
@@ -488,6 +604,12 @@ def run_ours(args, w):
         "clocks": clk,
         "device_status": status,
     }
+    if recs is not None:
+        line["per_config"] = _per_config_json(recs, clocks, peak, peak_sus)
+        line["per_config_note"] = (f"fa_fwd + fa_bwd steps of each causal configuration, each timed back to back "
+                                   f"for about {PER_CONFIG_SECONDS:g} s after 3 warm-up steps, with the clock "
+                                   "samples of its own timed window; *_frac use the peak those samples select "
+                                   "(peak_rule)")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = len(os.sched_getaffinity(0))
         heads = 4
@@ -668,6 +790,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=sorted(WORKLOADS) + sorted(EXTRA_WORKLOADS) + sorted(DECODE_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-configuration records (N = 2K, 8K, 32K, 128K) of the default workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -100,6 +100,12 @@ def _stream_ptr(t: torch.Tensor):
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
 
+def _on(t: torch.Tensor):
+    """Make t's device current for a library call: the library takes its SM count, kernel
+    set-up and status word from the current device, and launches on that device's stream."""
+    return torch.cuda.device(t.device)
+
+
 def validate_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not isinstance(t, torch.Tensor):
@@ -168,8 +174,9 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     check_buffer("lse", lse, (B, H, N), torch.float32, q.device)
     p = problem(q, k, causal, scale, window)
-    st = lib().fa_fwd_ex(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                         lse.data_ptr(), _stream_ptr(q))
+    with _on(q):
+        st = lib().fa_fwd_ex(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), _stream_ptr(q))
     if st != 0:
         raise FAError(st, "fa_fwd_ex")
     return out, lse
@@ -189,9 +196,10 @@ def fwd_e4m3(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_descale: float
     check_buffer("out", out, q.shape, torch.bfloat16, q.device)
     check_buffer("lse", lse, (B, H, N), torch.float32, q.device)
     p = problem(q, k, causal, scale, window)
-    st = lib().fa_fwd_e4m3_scaled(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                  float(q_descale), float(k_descale), float(v_descale), out.data_ptr(),
-                                  lse.data_ptr(), _stream_ptr(q))
+    with _on(q):
+        st = lib().fa_fwd_e4m3_scaled(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                      float(q_descale), float(k_descale), float(v_descale), out.data_ptr(),
+                                      lse.data_ptr(), _stream_ptr(q))
     if st != 0:
         raise FAError(st, "fa_fwd_e4m3_scaled")
     return out, lse
@@ -225,9 +233,10 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, do: 
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     check_scratch("workspace", workspace, q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
-    st = lib().fa_bwd_ex(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                         do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                         workspace.data_ptr(), ws_bytes, _stream_ptr(q))
+    with _on(q):
+        st = lib().fa_bwd_ex(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                             workspace.data_ptr(), ws_bytes, _stream_ptr(q))
     if st != 0:
         raise FAError(st, "fa_bwd_ex")
     return dq, dk, dv
@@ -243,8 +252,10 @@ def decode_problem(q: torch.Tensor, k_cache: torch.Tensor, causal: bool, scale: 
 
 def decode_workspace_size(q: torch.Tensor, k_cache: torch.Tensor, causal: bool = True,
                           window: int | None = None) -> int:
-    """Bytes of device workspace ``fa_decode`` needs for these shapes on the current device."""
-    return int(lib().fa_decode_workspace_size(ctypes.byref(decode_problem(q, k_cache, causal, None, window))))
+    """Bytes of device workspace ``fa_decode`` needs for these shapes on q's device (the split
+    depends on that device's SM count)."""
+    with _on(q):
+        return int(lib().fa_decode_workspace_size(ctypes.byref(decode_problem(q, k_cache, causal, None, window))))
 
 
 def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
@@ -276,23 +287,27 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     check_buffer("out", out, q.shape, q.dtype, q.device)
     check_buffer("lse", lse, (B, H, n_q), torch.float32, q.device)
     p = decode_problem(q, k_cache, causal, scale, window)
-    need = int(lib().fa_decode_workspace_size(ctypes.byref(p)))
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    check_scratch("workspace", workspace, q.device)
-    ws_bytes = workspace.numel() * workspace.element_size()
-    st = lib().fa_decode(ctypes.byref(p), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
-                         None if seqlens is None else seqlens.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                         workspace.data_ptr(), ws_bytes, _stream_ptr(q))
+    with _on(q):
+        need = int(lib().fa_decode_workspace_size(ctypes.byref(p)))
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+        check_scratch("workspace", workspace, q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+        st = lib().fa_decode(ctypes.byref(p), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                             None if seqlens is None else seqlens.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             workspace.data_ptr(), ws_bytes, _stream_ptr(q))
     if st != 0:
         raise FAError(st, "fa_decode")
     return out, lse
 
 
 def get_status(device: torch.device | None = None) -> int:
-    """Synchronise the current stream and read-and-clear the device status word."""
-    s = torch.cuda.current_stream(device)
-    return int(lib().fa_get_status(ctypes.c_void_p(s.cuda_stream)))
+    """Synchronise the device's current stream and read-and-clear that device's status word
+    (the current device when none is given)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev)
+        return int(lib().fa_get_status(ctypes.c_void_p(s.cuda_stream)))
 
 
 def selftest_wait_timeout(timeout_us: int = 20000) -> int:

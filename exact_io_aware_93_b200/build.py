@@ -10,6 +10,7 @@ only the NVIDIA driver at run time.
 from __future__ import annotations
 
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -45,6 +46,52 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
+# Kernels whose warpgroups rebalance registers with setmaxnreg: the split assumes that ptxas
+# gives every instantiation exactly the launch allocation named by the constant.
+REG_CONTRACT = {
+    "fa_fwd_kernel": ("fa_fwd_kernel.cuh", "kLaunchRegs"),
+    "fa_bwd_main_kernel": ("fa_bwd_kernel.cuh", "kBwdLaunchRegs"),
+}
+
+
+def _constant(header: str, name: str) -> int:
+    with open(os.path.join(CSRC, header)) as f:
+        m = re.search(r"constexpr\s+uint32_t\s+" + name + r"\s*=\s*(\d+)", f.read())
+    if not m:
+        raise RuntimeError(f"{name} not found in {header}")
+    return int(m.group(1))
+
+
+def ptxas_registers(log: str):
+    """(mangled entry name, registers) for every entry function in a `-Xptxas -v` report."""
+    out, current = [], None
+    for line in log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            current = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and current is not None:
+            out.append((current, int(m.group(1))))
+            current = None
+    return out
+
+
+def check_register_contract(log: str) -> None:
+    """Fail when a setmaxnreg kernel was compiled to a register count other than its launch
+    allocation: the warpgroups' register split would then not add up."""
+    regs = ptxas_registers(log)
+    bad = []
+    for kernel, (header, const) in REG_CONTRACT.items():
+        want = _constant(header, const)
+        found = [(name, n) for name, n in regs if kernel in name]
+        if not found:
+            bad.append(f"{kernel}: no instantiation in the ptxas report")
+        bad += [f"{name}: {n} registers, the split assumes {want}" for name, n in found if n != want]
+    if bad:
+        raise RuntimeError("register contract broken:\n  " + "\n  ".join(bad))
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB_PATH
@@ -58,6 +105,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
         f.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed (see {log}):\n{res.stderr[-4000:]}")
+    try:
+        check_register_contract(res.stdout + res.stderr)
+    except RuntimeError:
+        os.unlink(tmp)
+        raise
     os.replace(tmp, LIB_PATH)
     if verbose:
         print(res.stderr)

@@ -5,6 +5,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/fa.h"
@@ -20,8 +21,12 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Per-device set-up.  The first call on a device fills `ok`, `sm_count` and `status` under
+// g_dev_mutex and only then publishes `probed` (release); later calls read `probed`
+// (acquire) without the lock.  The kernel-attribute flags are set under the same mutex, so
+// first calls from several host threads at once are safe.
 struct DeviceInfo {
-  bool probed = false;
+  std::atomic<bool> probed{false};
   bool ok = false;
   int sm_count = 0;
   int* status = nullptr;
@@ -30,12 +35,28 @@ struct DeviceInfo {
   bool dec_attr[2][2][4] = {};  // [fp16][d==128][M = 128; M = 64 with 1, 2, 4 row copies]
 };
 DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+// Runs `setup` (which returns true on success) once per flag, under g_dev_mutex.
+template <typename F>
+bool once_per_device(bool& flag, F setup) {
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (!flag) {
+    if (!setup()) {
+      cudaGetLastError();
+      return false;
+    }
+    flag = true;
+  }
+  return true;
+}
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // The warp-specialised kernels move registers between warpgroups with setmaxnreg; the
-// split is computed for a launch at exactly fa::kLaunchRegs registers per thread.
-// Refuse to launch a build whose register count differs.
+// split is computed for a launch at exactly fa::kLaunchRegs registers per thread.  The
+// build script fails when ptxas reports another count; this check refuses to launch a
+// library that was built some other way with a different count.
 template <typename K>
 bool launch_regs_ok(K kern, uint32_t expected) {
   cudaFuncAttributes a;
@@ -53,20 +74,20 @@ fa_status current_device(DeviceInfo** out) {
     return FA_ERR_DEVICE;
   }
   DeviceInfo& di = g_dev[dev];
-  if (!di.probed) {
-    di.probed = true;
-    cudaDeviceProp prop;
-    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+  if (!di.probed.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!di.probed.load(std::memory_order_relaxed)) {
+      cudaDeviceProp prop;
+      void* sym = nullptr;
+      if (cudaGetDeviceProperties(&prop, dev) == cudaSuccess && prop.major == 10 && prop.minor == 0 &&
+          cudaGetSymbolAddress(&sym, g_fa_status) == cudaSuccess && sym != nullptr) {
+        di.ok = true;
+        di.sm_count = prop.multiProcessorCount;
+        di.status = static_cast<int*>(sym);
+      }
       cudaGetLastError();
-      return FA_ERR_DEVICE;
+      di.probed.store(true, std::memory_order_release);
     }
-    void* sym = nullptr;
-    if (prop.major == 10 && prop.minor == 0 && cudaGetSymbolAddress(&sym, g_fa_status) == cudaSuccess) {
-      di.ok = true;
-      di.sm_count = prop.multiProcessorCount;
-      di.status = static_cast<int*>(sym);
-    }
-    cudaGetLastError();
   }
   if (!di.ok) return FA_ERR_DEVICE;
   *out = &di;
@@ -101,15 +122,11 @@ fa_status launch_fwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   using T = typename fa::FwdOut<E>::T;
   auto kern = fa::fa_fwd_kernel<D, CAUSAL, E>;
   const int smem = static_cast<int>(sizeof(fa::FwdSmem<D, E>)) + 1024;
-  bool& attr = di.fwd_attr[static_cast<int>(E)][D == 128][CAUSAL];
-  if (!attr) {
-    if (!launch_regs_ok(kern, fa::kLaunchRegs) ||
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_LAUNCH;
-    }
-    attr = true;
-  }
+  if (!once_per_device(di.fwd_attr[static_cast<int>(E)][D == 128][CAUSAL], [&] {
+        return launch_regs_ok(kern, fa::kLaunchRegs) &&
+               cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+      }))
+    return FA_ERR_LAUNCH;
   const long long nkb = (static_cast<long long>(N) + 127) / 128;
   const long long tiles = static_cast<long long>(B) * H * ((nkb + 1) / 2);
   const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
@@ -140,22 +157,19 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + rows * D * 4);
   float* lse2 = dsum + prows;
   const unsigned pre_blocks = static_cast<unsigned>((prows * (D / 8) + 255) / 256);
-  fa::fa_bwd_pre_kernel<D, E><<<pre_blocks, 256, 0, stream>>>(static_cast<const T*>(o), static_cast<const T*>(dO),
-                                                              lse, dsum, lse2, dq_acc, B, H, N);
   const int64_t ew_threads = rows * (D / 8);
   const unsigned ew_blocks = static_cast<unsigned>((ew_threads + 255) / 256);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   auto kern = fa::fa_bwd_main_kernel<D, CAUSAL, E>;
   const int smem = static_cast<int>(sizeof(fa::BwdSmem<D>));
-  bool& attr = di.bwd_attr[E == fa::Elem::kF16][D == 128][CAUSAL];
-  if (!attr) {
-    if (!launch_regs_ok(kern, fa::kBwdLaunchRegs) ||
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_LAUNCH;
-    }
-    attr = true;
-  }
+  // every check that can fail comes before the first launch: on error nothing is enqueued
+  if (!once_per_device(di.bwd_attr[E == fa::Elem::kF16][D == 128][CAUSAL], [&] {
+        return launch_regs_ok(kern, fa::kBwdLaunchRegs) &&
+               cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+      }))
+    return FA_ERR_LAUNCH;
+  fa::fa_bwd_pre_kernel<D, E><<<pre_blocks, 256, 0, stream>>>(static_cast<const T*>(o), static_cast<const T*>(dO),
+                                                              lse, dsum, lse2, dq_acc, B, H, N);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   const int nkb = (N + 127) / 128;
   kern<<<B * H_kv * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, lse2, dsum, dq_acc, static_cast<T*>(dk),
                                                            static_cast<T*>(dv), B, H, H_kv, N, window, scale,
@@ -265,14 +279,10 @@ fa_status launch_decode(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap
                    : (R == 4 ? fa::fa_decode_kernel<D, E, 4, 64>
                              : (R == 2 ? fa::fa_decode_kernel<D, E, 2, 64> : fa::fa_decode_kernel<D, E, 1, 64>));
   const int smem = static_cast<int>(sizeof(fa::DecSmem<D>)) + 1024;
-  bool& attr = di.dec_attr[E == fa::Elem::kF16][D == 128][m64 ? 1 + (R >> 1) : 0];
-  if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_LAUNCH;
-    }
-    attr = true;
-  }
+  if (!once_per_device(di.dec_attr[E == fa::Elem::kF16][D == 128][m64 ? 1 + (R >> 1) : 0], [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+      }))
+    return FA_ERR_LAUNCH;
   const int grid = di.sm_count;
   const DecLayout L = dec_layout(p, grid);
   uint8_t* w = static_cast<uint8_t*>(ws);

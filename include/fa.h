@@ -177,7 +177,9 @@ fa_status fa_bwd_ex(const fa_problem* problem, const void* q, const void* k, con
  * another allocator, or where the implicit synchronisation of cudaMalloc / cudaFree is
  * not acceptable.  (The pages describe no such entry point; it has no counterpart there.)
  * It performs the same computation as fa_bwd, with the same arguments minus the
- * workspace, and calls no cudaMalloc, cudaFree or other allocating routine.
+ * workspace, and calls no cudaMalloc, cudaFree or other allocating routine.  Like fa_bwd
+ * it covers bf16 tensors with H_kv == H and no sliding window only; fp16, grouped-query
+ * and windowed problems go through fa_bwd_ex with a caller-provided workspace.
  *
  * Scratch: a fixed 64 MiB array inside the library holding what fa_bwd's workspace would
  * (fa_bwd_workspace_size bytes).  Problems that need more return FA_ERR_WORKSPACE and launch

@@ -56,3 +56,47 @@ def test_traffic_only_for_matching_sources(tmp_path, monkeypatch):
 def test_source_digest_is_stable():
     assert bench.kernel_source_digest() == bench.kernel_source_digest()
     assert len(bench.kernel_source_digest()) == 16
+
+
+# nvidia-smi rows in the order of ClockSampler.QUERY
+_ROW = "{ts}, 0, {sm} MHz, 1965 MHz, {pw} W, 0x0, Not Active, Not Active, Not Active, {cap}"
+
+
+def _rows(specs):
+    return [_ROW.format(ts=ts, sm=sm, pw=pw, cap="Active" if cap else "Not Active") for ts, sm, pw, cap in specs]
+
+
+def test_clock_samples_parse_and_window():
+    rows = _rows([("2026/12/02 10:00:00.000", 1965, 300, False),
+                  ("2026/12/02 10:00:00.200", 1800, 900, True),
+                  ("2026/12/02 10:00:01.000", 1500, 1000, True)])
+    samples = bench.parse_clock_samples(rows + ["garbage", ""])
+    assert len(samples) == 3
+    assert samples[1]["reasons"] == ["sw_power_cap"] and samples[0]["reasons"] == []
+    t0 = samples[0]["ts"]
+    st = bench.clock_stats(samples, (t0, t0 + 0.3))
+    assert st["samples"] == 2 and st["power_cap_samples"] == 1
+    assert st["sm_mhz"] == (1965 + 1800) / 2 and st["sm_max_mhz"] == 1965 and st["power_w_max"] == 900
+    assert st["reasons"] == ["sw_power_cap"]
+    assert bench.clock_stats(samples, (t0 + 5, t0 + 6))["samples"] == 0
+
+
+def test_peak_follows_the_regions_own_clock_samples():
+    burst, sus = 1652.2, 1379.2
+    # no in-region sample saw the power cap: burst peak, and the rule says on how many samples
+    peak, kind, rule = bench.choose_peak({"samples": 3, "power_cap_samples": 0}, burst, sus)
+    assert (peak, kind) == (burst, "burst") and "0 of 3" in rule
+    # one capped sample is enough for the sustained peak
+    peak, kind, rule = bench.choose_peak({"samples": 4, "power_cap_samples": 1}, burst, sus)
+    assert (peak, kind) == (sus, "sustained") and "1 of 4" in rule
+    # no samples at all: the burst peak (the larger denominator, so the smaller fraction)
+    peak, kind, _ = bench.choose_peak({"samples": 0, "power_cap_samples": 0}, burst, sus)
+    assert peak == burst
+
+
+def test_per_config_covers_the_metrics_range():
+    from exact_io_aware_93_b200.inputs import WORKLOADS
+    ns = sorted(WORKLOADS[n].N for n in bench.PER_CONFIG)
+    assert ns == [2048, 8192, 32768, 131072]
+    assert all(WORKLOADS[n].causal for n in bench.PER_CONFIG)
+    assert bench.DEFAULT_WORKLOAD in bench.PER_CONFIG

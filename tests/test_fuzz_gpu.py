@@ -7,7 +7,7 @@ import torch
 
 from exact_io_aware_93_b200 import api
 from exact_io_aware_93_b200.inputs import make_decode_inputs, make_inputs
-from tests.parity import GRAD_TOL, LSE_TOL, O_TOL, decode_errors, fwd_errors_gqa, grad_errors_gqa
+from tests.parity import GRAD_TOL, LSE_TOL, O_TOL, decode_errors, fwd_errors, fwd_errors_gqa, grad_errors_gqa
 
 pytestmark = pytest.mark.gpu
 
@@ -35,7 +35,13 @@ def test_fuzz_fwd_bwd(seed):
     dq, dk, dv = api.bwd(q, k, v, o, do, lse, causal=c["causal"], window=w)
     torch.cuda.synchronize()
     assert api.get_status() == 0, c
-    eo, el = fwd_errors_gqa(inp, o, lse, c["d"] ** -0.5, c["causal"], c["window"])
+    if c["H_kv"] == c["H"] and c["window"] < 0:
+        # plain multi-head attention: the five configurations' gate, max |O - O_ref| itself
+        eo, el, where = fwd_errors(inp, o, lse, c["d"] ** -0.5, c["causal"])
+    else:
+        # grouped heads or a window: rows may see one or two keys, where the output's own
+        # rounding reaches 1e-2; judged by the excess over half an ulp (tests/parity.py)
+        eo, el = fwd_errors_gqa(inp, o, lse, c["d"] ** -0.5, c["causal"], c["window"])
     assert eo <= O_TOL and el <= LSE_TOL, (c, eo, el)
     err = grad_errors_gqa(inp, {"dq": dq.cpu(), "dk": dk.cpu(), "dv": dv.cpu()}, c["d"] ** -0.5, c["causal"],
                           c["window"])
