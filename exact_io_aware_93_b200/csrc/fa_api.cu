@@ -162,6 +162,8 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
   auto kern = fa::fa_bwd_main_kernel<D, CAUSAL, E>;
   const int smem = static_cast<int>(sizeof(fa::BwdSmem<D>));
   // every check that can fail comes before the first launch: on error nothing is enqueued
+  CUtensorMap mdq;  // the fp32 dQ accumulator, target of the main kernel's TMA reduce-adds
+  if (!fa::make_dqacc_map(&mdq, dq_acc, static_cast<long long>(B) * H, N, D)) return FA_ERR_LAUNCH;
   if (!once_per_device(di.bwd_attr[E == fa::Elem::kF16][D == 128][CAUSAL], [&] {
         return launch_regs_ok(kern, fa::kBwdLaunchRegs) &&
                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
@@ -171,7 +173,7 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
                                                               lse, dsum, lse2, dq_acc, B, H, N);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   const int nkb = (N + 127) / 128;
-  kern<<<B * H_kv * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, lse2, dsum, dq_acc, static_cast<T*>(dk),
+  kern<<<B * H_kv * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, mdq, lse2, dsum, static_cast<T*>(dk),
                                                            static_cast<T*>(dv), B, H, H_kv, N, window, scale,
                                                            di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;

@@ -21,28 +21,34 @@
 //                   dS^T = P^T o (dP^T - D_i)   (with the bf16 P^T that enters dV)
 //                   dV_j += P^T dO_i        (A operand P^T read from tensor memory)
 //                   dK_j += dS^T Q_i        (A operand dS^T read from shared memory)
-//                   dQ_i  = dS K_j          (dS written to shared memory, 128-byte swizzle);
-//                                           for d = 128 computed transposed, dQ_i^T = K_j^T dS^T,
-//                                           so that tensor-memory lanes are head-dim columns
+//                   dQ_i  = dS K_j          (dS written to shared memory, 128-byte swizzle;
+//                                           tensor-memory lanes are query rows)
 //                 and a drain warpgroup copies each dQ_i tile out of tensor memory, frees it,
-//                 and adds it into the fp32 accumulator with reductions that cover whole
-//                 128-byte lines; dK_j, dV_j accumulate over the whole group in tensor
-//                 memory and are written once at the end.
+//                 stages its rows in shared memory and adds them into the fp32 accumulator
+//                 with TMA reduce-adds (one bulk operation per 32 rows x 32 columns, issued
+//                 by one thread, instead of a reduction instruction per element); dK_j, dV_j
+//                 accumulate over the whole group in tensor memory and are written once at
+//                 the end.
 //   Per query block the MMA warp issues dP, then (once P is ready) dV and the next block's
-//   S, then (once dS is ready) dK and dQ, so the tensor core works while the key-row
-//   warpgroups compute dS and while the drain empties the previous dQ tile.
+//   S, then (once dS is ready) dK and dQ interleaved (two independent accumulators), so the
+//   tensor core works while the key-row warpgroups compute dS and while the drain empties
+//   the previous dQ tile.
 //   fa_bwd_post : dQ = bf16(scale * accumulator)
 //
 // Tensor memory (512 columns):
 //   [0,128)   S^T  (fp32).  Key-row warpgroup g (queries 64g..64g+63) reads columns
 //             [64g, 64g+64) and writes its bf16 P^T into [64g, 64g+32), inside its own range.
-//   [128,256) dP^T (fp32); once the key rows have read it, dQ_i (or dQ_i^T), fp32
+//   [128,128+D) dP^T (fp32); once the key rows have read it, dQ_i (query rows on lanes), fp32
 //   [256,256+D) dV_j accumulator,  [384,384+D) dK_j accumulator
 //
+// Shared memory: K_j, V_j; Q_i in a two-stage ring together with the block's LSE * log2 e
+// and D runs; dO_i in one buffer (it is read only by the dP and dV products, early in the
+// block, and is reloaded while the rest of the block runs); dS; two 32-row dQ staging slots.
+//
 // Warp roles (512 threads): warps 0-3 and 4-7 key rows for queries 0-63 and 64-127 of the
-// block (P, dS; at the end dV and dK respectively), warps 8-11 dQ drain, warp 12 loads (TMA
-// tiles for Q, dO and bulk copies of the block's LSE * log2 e and D), warp 13 issues MMAs,
-// warps 14-15 idle.
+// block (P, dS; at the end dV and dK respectively), warps 8-11 dQ drain (warp 8 + w holds
+// query rows 32w..32w+31), warp 12 loads (TMA tiles for Q, dO and bulk copies of the
+// block's LSE * log2 e and D), warp 13 issues MMAs, warps 14-15 idle.
 #pragma once
 
 #include "fa_fwd_kernel.cuh"
@@ -54,7 +60,7 @@ constexpr int kBwdThreads = 512;
 constexpr uint32_t kBwdLaunchRegs = 128;  // 65536 / 512
 constexpr uint32_t kBwdRegsKey = 112;     // two key-row warpgroups
 constexpr uint32_t kBwdRegsDrain = 168;
-constexpr uint32_t kBwdRegsOther = 96;
+constexpr uint32_t kBwdRegsOther = 104;
 static_assert(128 * (2 * kBwdRegsKey + kBwdRegsDrain + kBwdRegsOther) <= kBwdThreads * kBwdLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr float kLog2e = 1.4426950408889634f;
@@ -68,6 +74,7 @@ struct BwdCfg {
   static constexpr uint32_t kColDP = 128;
   static constexpr uint32_t kColDV = 256;
   static constexpr uint32_t kColDK = 384;
+  static constexpr int kStageBytes = 32 * D * 4;  // one drain warp's 32 rows of dQ
 };
 
 template <int D>
@@ -75,13 +82,19 @@ struct __align__(1024) BwdSmem {
   uint8_t k[BwdCfg<D>::kTileBytes];
   uint8_t v[BwdCfg<D>::kTileBytes];
   uint8_t q[2][BwdCfg<D>::kTileBytes];
-  uint8_t dO[2][BwdCfg<D>::kTileBytes];
+  uint8_t dO[BwdCfg<D>::kTileBytes];
   uint8_t ds[128 * 128 * 2];  // dS (queries x keys), MN-major A operand of dQ = dS K
+  // dQ staging: two slots of 32 query rows x D fp32, each as D/32 boxes of 32 rows x 128
+  // bytes in the 128-byte swizzle of the accumulator's tensor map
+  uint8_t stg[2][BwdCfg<D>::kStageBytes];
   float lse2[2][128];         // LSE * log2(e) of the query block (+inf past the sequence)
   float dd[2][128];           // D of the query block
   uint64_t kv_full;
-  uint64_t qd_full[2];
-  uint64_t qd_empty[2];
+  uint64_t q_full[2];
+  uint64_t q_empty[2];
+  uint64_t do_full;
+  uint64_t do_empty;
+  uint64_t stg_free[2];
   uint64_t s_full;
   uint64_t dp_full;
   uint64_t p_ready;
@@ -165,15 +178,6 @@ __global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restric
   *reinterpret_cast<uint4*>(dq + ((static_cast<int64_t>(b) * N + n) * H + h) * D + part * 8) = r;
 }
 
-__device__ __forceinline__ void red_add(float* addr, float a) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
-}
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
 // P^T for 32 queries of one key row: p = 2^(s * sl - lse2), zero where masked
 // (MASKED: key beyond the sequence, query index below qlim on the diagonal block, or above
 // qhi past the end of a sliding window);
@@ -210,8 +214,8 @@ template <int D, bool CAUSAL, Elem E = Elem::kBf16>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                       const float* __restrict__ lse2g, const float* __restrict__ dsum,
-                       float* __restrict__ dq_acc, typename ElemOps<E>::T* __restrict__ dk,
+                       const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ lse2g,
+                       const float* __restrict__ dsum, typename ElemOps<E>::T* __restrict__ dk,
                        typename ElemOps<E>::T* __restrict__ dv,
                        int B, int H, int H_kv, int N, int window, float scale, int* status) {
   using Cfg = BwdCfg<D>;
@@ -247,9 +251,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     sm.abort_flag = 0;
     mbar_init(&sm.kv_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.qd_full[s], 1);
-      mbar_init(&sm.qd_empty[s], 1);
+      mbar_init(&sm.q_full[s], 1);
+      mbar_init(&sm.q_empty[s], 1);
+      mbar_init(&sm.stg_free[s], 1);
     }
+    mbar_init(&sm.do_full, 1);
+    mbar_init(&sm.do_empty, 1);
     mbar_init(&sm.s_full, 1);
     mbar_init(&sm.dp_full, 1);
     mbar_init(&sm.p_ready, 256);
@@ -281,6 +288,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_dq);
       mbar_arrive_expect_tx(&sm.kv_full, 2 * Cfg::kTileBytes);
       for (int c = 0; c < Cfg::kChunks; ++c) {
         tma_load_4d(sm.k + c * Cfg::kChunkBytes, &tm_k, &sm.kv_full, c * 64, hkv, j * 128, b);
@@ -288,32 +296,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     const int npad = nkb * 128;
-    int issued = 0;
+    int q_issued = 0, do_issued = 0;
     bool ok = true;
+    // Q_i (ring stage idx & 1, freed by the block's dK product) and dO_i (one buffer, freed
+    // by the previous block's dV product) are issued in this order, which is also the order
+    // in which their buffers free up.
     for (int idx = 0; idx < ni; ++idx) {
       const int st = idx & 1;
       const int i = i0 + idx % nper;
       const int h = hkv * group + idx / nper;
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.qd_empty[st], ((idx >> 1) & 1) ^ 1, wc));
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_empty[st], ((idx >> 1) & 1) ^ 1, wc));
+      if (!ok) break;
+      const int64_t ridx = (static_cast<int64_t>(b) * H + h) * npad + i * 128;
+      if (lane == 0) {
+        // Q_i tile plus the block's LSE2 and D runs (512 bytes each, padded rows)
+        mbar_arrive_expect_tx(&sm.q_full[st], Cfg::kTileBytes + 2 * 512);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_4d(sm.q[st] + c * Cfg::kChunkBytes, &tm_q, &sm.q_full[st], c * 64, h, i * 128, b);
+        bulk_load(sm.lse2[st], lse2g + ridx, 512, &sm.q_full[st]);
+        bulk_load(sm.dd[st], dsum + ridx, 512, &sm.q_full[st]);
+      }
+      ++q_issued;
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.do_empty, (idx & 1) ^ 1, wc));
       if (!ok) break;
       if (lane == 0) {
-        // Q_i, dO_i tiles plus the block's LSE2 and D runs (512 bytes each, padded rows)
-        mbar_arrive_expect_tx(&sm.qd_full[st], 2 * Cfg::kTileBytes + 2 * 512);
-        for (int c = 0; c < Cfg::kChunks; ++c) {
-          tma_load_4d(sm.q[st] + c * Cfg::kChunkBytes, &tm_q, &sm.qd_full[st], c * 64, h, i * 128, b);
-          tma_load_4d(sm.dO[st] + c * Cfg::kChunkBytes, &tm_do, &sm.qd_full[st], c * 64, h, i * 128, b);
-        }
-        const int64_t ridx = (static_cast<int64_t>(b) * H + h) * npad + i * 128;
-        bulk_load(sm.lse2[st], lse2g + ridx, 512, &sm.qd_full[st]);
-        bulk_load(sm.dd[st], dsum + ridx, 512, &sm.qd_full[st]);
+        mbar_arrive_expect_tx(&sm.do_full, Cfg::kTileBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_4d(sm.dO + c * Cfg::kChunkBytes, &tm_do, &sm.do_full, c * 64, h, i * 128, b);
       }
-      ++issued;
+      ++do_issued;
     }
     if (!ok && lane == 0) {
       // unwinding: wait (bounded) for the copies in flight
       mbar_wait_drain(&sm.kv_full, 0, status);
-      for (int idx = (issued > 2 ? issued - 2 : 0); idx < issued; ++idx)
-        mbar_wait_drain(&sm.qd_full[idx & 1], (idx >> 1) & 1, status);
+      for (int idx = (q_issued > 2 ? q_issued - 2 : 0); idx < q_issued; ++idx)
+        mbar_wait_drain(&sm.q_full[idx & 1], (idx >> 1) & 1, status);
+      if (do_issued > 0) mbar_wait_drain(&sm.do_full, (do_issued - 1) & 1, status);
     }
   } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
@@ -338,24 +356,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           umma_ss(tD, da + off, db + off, idesc_sdp, kk > 0);
         }
       };
-      constexpr bool kDqT = (D == 128);  // dQ^T = K^T dS^T: M = d, N = 128 queries
-      constexpr uint32_t idesc_dqt = idesc_kind_f16(128, 128, 1, 1, kT);
-      bool ok = mbar_wait(&sm.kv_full, 0, wc) && mbar_wait(&sm.qd_full[0], 0, wc);
+      bool ok = mbar_wait(&sm.kv_full, 0, wc) && mbar_wait(&sm.q_full[0], 0, wc);
       if (ok) {
         tc_fence_after();
         kmaj_gemm(tS, dk_kmaj, sdesc_sw128(smem_u32(sm.q[0]), 16, 1024));  // S^T for the first block
         umma_commit(&sm.s_full);
       }
+      const uint64_t ddo_k = sdesc_sw128(smem_u32(sm.dO), 16, 1024);
+      const uint64_t ddo_mn = sdesc_sw128(smem_u32(sm.dO), Cfg::kChunkBytes, 1024);
       for (int idx = 0; idx < ni && ok; ++idx) {
         const int st = idx & 1;
-        const uint64_t ddo_k = sdesc_sw128(smem_u32(sm.dO[st]), 16, 1024);
         const uint64_t dq_mn = sdesc_sw128(smem_u32(sm.q[st]), Cfg::kChunkBytes, 1024);
-        const uint64_t ddo_mn = sdesc_sw128(smem_u32(sm.dO[st]), Cfg::kChunkBytes, 1024);
         if (idx > 0) {
           ok = mbar_wait(&sm.dq_free, (idx - 1) & 1, wc);  // dQ_{i-1} copied out of the dP columns
           if (!ok) break;
-          tc_fence_after();
         }
+        ok = mbar_wait(&sm.do_full, idx & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
         kmaj_gemm(tDP, dv_kmaj, ddo_k);  // dP^T = V dO^T
         umma_commit(&sm.dp_full);
         ok = mbar_wait(&sm.p_ready, idx & 1, wc);
@@ -366,8 +384,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, ddo_mn + ((kk * 2048) >> 4), idesc_acc,
                   (kk > 0) || (idx > 0));
         }
+        umma_commit(&sm.do_empty);  // dO_i is no longer read once dP and dV complete
         if (idx + 1 < ni) {  // next block's S^T, into the columns P^T just left
-          ok = mbar_wait(&sm.qd_full[st ^ 1], ((idx + 1) >> 1) & 1, wc);
+          ok = mbar_wait(&sm.q_full[st ^ 1], ((idx + 1) >> 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
           kmaj_gemm(tS, dk_kmaj, sdesc_sw128(smem_u32(sm.q[st ^ 1]), 16, 1024));
@@ -376,20 +395,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = mbar_wait(&sm.ds_ready, idx & 1, wc);
         if (!ok) break;
         tc_fence_after();
+        // dK += dS^T Q (dS^T read K-major from shared memory) and dQ = dS K (K = 128 keys, into
+        // the dP columns), interleaved: two independent accumulators keep the tensor core full
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q, dS^T read K-major from shared memory
+        for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4;
           umma_ss(tDK, dds_k + off, dq_mn + ((kk * 2048) >> 4), idesc_acc, (kk > 0) || (idx > 0));
+          umma_ss(tDP, dds + ((kk * 2048) >> 4), dk_mn + ((kk * 2048) >> 4), idesc_dq, kk > 0);
         }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // dQ (K = 128 keys) into the dP columns
-          if constexpr (kDqT)
-            umma_ss(tDP, dk_mn + ((kk * 2048) >> 4), dds + ((kk * 2048) >> 4), idesc_dqt, kk > 0);
-          else
-            umma_ss(tDP, dds + ((kk * 2048) >> 4), dk_mn + ((kk * 2048) >> 4), idesc_dq, kk > 0);
-        }
+        umma_commit(&sm.q_empty[st]);
         umma_commit(&sm.dq_full);
-        umma_commit(&sm.qd_empty[st]);
       }
       umma_commit(&sm.acc_done);
       umma_commit(&sm.mma_drain);
@@ -414,7 +429,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int idx = 0; idx < ni && ok; ++idx) {
       const int st = idx & 1;
       const int i = i0 + idx % nper;
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.qd_full[st], (idx >> 1) & 1, wc));
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full[st], (idx >> 1) & 1, wc));
       ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.s_full, idx & 1, wc));
       if (!ok) break;
       tc_fence_after();
@@ -522,50 +537,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_before();
   } else {
     // ------------------------------------------------------------ dQ drain (warps 8-11)
+    // Warp 8 + w copies query rows 32w..32w+31 of dQ_i out of tensor memory, frees the
+    // columns, writes the rows into its staging slot in the 128-byte swizzle of the
+    // accumulator's tensor map, and one lane adds the slot into the fp32 accumulator with
+    // D/32 TMA reduce-adds (rows past the sequence fall outside the map and are skipped).
+    // Warps w and w + 2 share slot w & 1 and take turns: each waits until the other's
+    // reduce-adds have finished reading the slot (stg_free).
     regs_set<kBwdLaunchRegs, kBwdRegsDrain>();
-    const int r = threadIdx.x - 256;  // TMEM lane: head-dim column (d = 128) or query row (d = 64)
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int w = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(w * 32) << 16;
     const uint32_t tQ = tbase + Cfg::kColDP + lane_off;
+    const int slot = w & 1;
+    uint8_t* stg = sm.stg[slot];
+    uint8_t* my_row = stg + lane * 128;  // this lane's row inside each 32-row box
     const WaitCtx wc{&sm.abort_flag, status, 14};
     for (int idx = 0; idx < ni; ++idx) {
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, idx & 1, wc));
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, idx & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      const int q0 = (i0 + idx % nper) * 128;
-      const int64_t bh = static_cast<int64_t>(b) * H + hkv * group + idx / nper;  // query head row
-      if constexpr (D == 128) {
-        // lane r holds column r of dQ_i for the 128 queries; a warp's reduction for one query
-        // covers 32 consecutive columns = one 128-byte line
-        uint32_t a[128];
-        tmem_ld32(tQ + 0, a);
-        tmem_ld32(tQ + 32, a + 32);
-        tmem_ld32(tQ + 64, a + 64);
-        tmem_ld32(tQ + 96, a + 96);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&sm.dq_free);  // the dP columns may be overwritten from here on
-        const int qn = min(128, N - q0);
-        float* dst = dq_acc + (bh * N + q0) * D + r;
+      uint32_t a[D];
 #pragma unroll
-        for (int q = 0; q < 128; ++q)
-          if (q < qn) red_add(dst + static_cast<int64_t>(q) * D, __uint_as_float(a[q]));
-      } else {
-        const int qg = q0 + r;
-        float* dst = dq_acc + (bh * N + qg) * D;
-        uint32_t a[D];
-#pragma unroll
-        for (int c = 0; c < D; c += 32) tmem_ld32(tQ + c, a + c);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&sm.dq_free);
-        if (qg < N) {
-#pragma unroll
-          for (int x = 0; x < D; x += 4)
-            red_add_v4(dst + x, __uint_as_float(a[x]), __uint_as_float(a[x + 1]), __uint_as_float(a[x + 2]),
-                       __uint_as_float(a[x + 3]));
-        }
+      for (int c = 0; c < D; c += 32) tmem_ld32(tQ + c, a + c);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&sm.dq_free);  // the dP columns may be overwritten from here on
+      // The slot's users alternate: warp w at block idx is user 2 idx, warp w + 2 user
+      // 2 idx + 1; user k waits for the k-th arrival, i.e. for the phase of parity (k-1) & 1.
+      if (w >= 2 || idx > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.stg_free[slot], w >= 2 ? 0u : 1u, wc));
+        if (!ok) break;
       }
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u)  // 16-byte unit u of the row lands at unit u ^ (row & 7)
+          *reinterpret_cast<uint4*>(my_row + c * 4096 + ((u ^ (lane & 7)) << 4)) =
+              make_uint4(a[32 * c + 4 * u], a[32 * c + 4 * u + 1], a[32 * c + 4 * u + 2], a[32 * c + 4 * u + 3]);
+      }
+      fence_proxy_async_smem();  // the generic-proxy stores become visible to the TMA unit
+      __syncwarp();
+      if (lane == 0) {
+        const int q0 = (i0 + idx % nper) * 128 + 32 * w;
+        const int bh = b * H + hkv * group + idx / nper;  // query head: row block of the accumulator
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tma_reduce_add_3d(&tm_dq, stg + c * 4096, 32 * c, q0, bh);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        mbar_arrive(&sm.stg_free[slot]);
+      }
+      __syncwarp();
     }
+    if (lane == 0) bulk_wait_group0();  // every reduce-add has landed before the CTA exits
   }
 
   tc_fence_before();

@@ -71,4 +71,20 @@ inline bool make_decode_q_map(CUtensorMap* map, const void* base, int B, int N_q
   return r == CUDA_SUCCESS;
 }
 
+// The backward's fp32 dQ accumulator [B*H, N, d] as a 3-D map {d, N, B*H} for TMA
+// reduce-adds from shared memory: boxes of 32 rows x 32 columns (128 bytes, 128-byte
+// swizzle).  Rows at or past N lie outside the map and are not written.
+inline bool make_dqacc_map(CUtensorMap* map, void* base, long long BH, int N, int d) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)N * d * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace fa
