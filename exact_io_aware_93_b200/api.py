@@ -22,7 +22,7 @@ _lib = None
 
 FA_STATUS = {
     0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_ALIGNMENT",
-    4: "FA_ERR_DEVICE", 5: "FA_ERR_LAUNCH", 6: "FA_ERR_TIMEOUT", 7: "FA_ERR_WORKSPACE",
+    4: "FA_ERR_DEVICE", 5: "FA_ERR_LAUNCH", 6: "FA_ERR_TIMEOUT", 7: "FA_ERR_WORKSPACE", 8: "FA_ERR_BOUNDS",
 }
 
 

@@ -19,6 +19,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB_NAME = "libfa_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
+# the same sources compiled with FA_CHECKS: every kernel bounds-checks its TMA coordinates
+# and global indices and reports a violation in the device status word (include/fa.h)
+CHECKS_LIB_PATH = os.path.join(PKG, "libfa_b200_checks.so")
 SOURCES = ["fa_api.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -39,10 +42,10 @@ def _deps():
     return out
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
+def up_to_date(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return False
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
@@ -92,15 +95,13 @@ def check_register_contract(log: str) -> None:
         raise RuntimeError("register contract broken:\n  " + "\n  ".join(bad))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB_PATH
-    tmp = f"{LIB_PATH}.{os.getpid()}.tmp"
+def _build_one(path: str, defines, log_name: str, verbose: bool) -> None:
+    tmp = f"{path}.{os.getpid()}.tmp"
     cmd = [_nvcc(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
-           "-Xptxas", "-v", "-cudart", "static",
+           "-Xptxas", "-v", "-cudart", "static", *defines,
            *[os.path.join(CSRC, s) for s in SOURCES], "-o", tmp]
     res = subprocess.run(cmd, capture_output=True, text=True)
-    log = os.path.join(PKG, "build.log")
+    log = os.path.join(PKG, log_name)
     with open(log, "w") as f:
         f.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
     if res.returncode != 0:
@@ -110,9 +111,18 @@ def build(force: bool = False, verbose: bool = False) -> str:
     except RuntimeError:
         os.unlink(tmp)
         raise
-    os.replace(tmp, LIB_PATH)
+    os.replace(tmp, path)
     if verbose:
         print(res.stderr)
+
+
+def build(force: bool = False, verbose: bool = False, checks: bool = True) -> str:
+    """Build the release library and (checks=True) the checking build; returns the release
+    library's path."""
+    if force or not up_to_date(LIB_PATH):
+        _build_one(LIB_PATH, [], "build.log", verbose)
+    if checks and (force or not up_to_date(CHECKS_LIB_PATH)):
+        _build_one(CHECKS_LIB_PATH, ["-DFA_CHECKS"], "build_checks.log", verbose)
     return LIB_PATH
 
 

@@ -170,14 +170,15 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
       }))
     return FA_ERR_LAUNCH;
   fa::fa_bwd_pre_kernel<D, E><<<pre_blocks, 256, 0, stream>>>(static_cast<const T*>(o), static_cast<const T*>(dO),
-                                                              lse, dsum, lse2, dq_acc, B, H, N);
+                                                              lse, dsum, lse2, dq_acc, B, H, N, di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   const int nkb = (N + 127) / 128;
   kern<<<B * H_kv * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, mdq, lse2, dsum, static_cast<T*>(dk),
                                                            static_cast<T*>(dv), B, H, H_kv, N, window, scale,
                                                            di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
-  fa::fa_bwd_post_kernel<D, E><<<ew_blocks, 256, 0, stream>>>(dq_acc, static_cast<T*>(dq), B, H, N, scale);
+  fa::fa_bwd_post_kernel<D, E><<<ew_blocks, 256, 0, stream>>>(dq_acc, static_cast<T*>(dq), B, H, N, scale,
+                                                               di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
 }
@@ -252,6 +253,7 @@ size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct DecLayout {
   size_t meta, part_lse, part_o, total;
+  size_t slots;  // partial results S = R * (grid + B * H_kv - 1)
 };
 
 // Workspace regions: schedule (total, tiles per CTA, per-sequence prefix), then the
@@ -263,6 +265,7 @@ DecLayout dec_layout(const fa_decode_problem& p, int grid) {
   const size_t slots = (static_cast<size_t>(grid) + static_cast<size_t>(p.B) * p.H_kv - 1) *
                        static_cast<size_t>(fa::dec_copies(static_cast<int>(M)));
   DecLayout L;
+  L.slots = slots;
   L.meta = 0;
   L.part_lse = round256((2 + static_cast<size_t>(p.B)) * 4);
   L.part_o = L.part_lse + round256(slots * M * 2 * 4);
@@ -304,6 +307,8 @@ fa_status launch_decode(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap
   a.causal = p.causal;
   a.R = R;
   a.scale_log2 = p.scale * 1.4426950408889634f;
+  a.slots = static_cast<long long>(L.slots);
+  a.status = di.status;
   kern<<<grid, fa::kDecThreads, smem, stream>>>(mq, mk, mv, a, di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   fa::fa_decode_merge_kernel<D, E><<<p.B * p.H_kv, 128, 0, stream>>>(a);
@@ -326,6 +331,18 @@ __global__ void fa_wait_timeout_selftest_kernel(uint64_t timeout_ns, int* status
   __syncwarp();
   const fa::WaitCtx wc{&abort_flag, status, 99};
   fa::mbar_wait(&bar, 0, wc, timeout_ns);
+}
+
+// ---------------------------------------------------------------- bounds-check self-test
+// One warp checks an index against a one-element target; lane 0's index is one past the
+// end, so in the checking build its check fails, records FA_ERR_BOUNDS and skips the store.
+// The array has a spare second element, so no build ever writes outside it.
+__global__ void fa_bounds_selftest_kernel(int* status) {
+  __shared__ int target[2];
+  const int idx = threadIdx.x == 0 ? 1 : 0;
+  if (FA_IN_BOUNDS(idx < 1, status, 999)) target[idx] = static_cast<int>(threadIdx.x);
+  __syncwarp();
+  (void)target[0];
 }
 
 // ---------------------------------------------------------------- allocation-free backward
@@ -369,7 +386,15 @@ fa_status noalloc_scratch(void** out) {
 
 extern "C" {
 
-int fa_abi_version(void) { return 4; }
+int fa_abi_version(void) { return 5; }
+
+int fa_checks_enabled(void) {
+#ifdef FA_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 const char* fa_status_string(int s) {
   switch (s) {
@@ -381,6 +406,7 @@ const char* fa_status_string(int s) {
     case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_BOUNDS: return "FA_ERR_BOUNDS";
     default: return "FA_ERR_UNKNOWN";
   }
 }
@@ -548,6 +574,19 @@ fa_status fa_selftest_wait_timeout(unsigned int timeout_us, void* stream) {
   fa_wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<uint64_t>(timeout_us) * 1000u, di->status);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+fa_status fa_selftest_bounds(void* stream) {
+#ifndef FA_CHECKS
+  (void)stream;
+  return FA_ERR_UNSUPPORTED;
+#else
+  DeviceInfo* di = nullptr;
+  const fa_status st = current_device(&di);
+  if (st != FA_OK) return st;
+  fa_bounds_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(di->status);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+#endif
 }
 
 fa_status fa_get_status(void* stream) {

@@ -118,7 +118,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const typename ElemOps<
                                                          const typename ElemOps<E>::T* __restrict__ dout,
                                                          const float* __restrict__ lse,
                                                          float* __restrict__ dsum, float* __restrict__ lse2,
-                                                         float* __restrict__ dq_acc, int B, int H, int N) {
+                                                         float* __restrict__ dq_acc, int B, int H, int N,
+                                                         int* status) {
   constexpr int TPR = D / 8;  // threads per row
   const int npad = (N + 127) / 128 * 128;
   const int64_t rows = static_cast<int64_t>(B) * H * npad;
@@ -131,6 +132,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const typename ElemOps<
   if (live) {
     const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
     const int64_t off = ((static_cast<int64_t>(b) * N + n) * H + h) * D + part * 8;
+    const int64_t elems = static_cast<int64_t>(B) * N * H * D;
+    if (!FA_IN_BOUNDS(off >= 0 && off + 8 <= elems && (bh * N + n) * D + part * 8 + 8 <= elems, status, 201)) return;
     const uint4 ov = *reinterpret_cast<const uint4*>(o + off);
     const uint4 dv = *reinterpret_cast<const uint4*>(dout + off);
     const uint32_t* op = reinterpret_cast<const uint32_t*>(&ov);
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const typename ElemOps<
   }
 #pragma unroll
   for (int s = TPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (row < rows && part == 0) {
+  if (row < rows && part == 0 && FA_IN_BOUNDS(row >= 0 && bh < static_cast<int64_t>(B) * H, status, 202)) {
     dsum[row] = live ? acc : 0.f;
     lse2[row] = live ? lse[bh * N + n] * 1.4426950408889634f : INFINITY;
   }
@@ -159,7 +162,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const typename ElemOps<
 template <int D, Elem E = Elem::kBf16>
 __global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restrict__ dq_acc,
                                                           typename ElemOps<E>::T* __restrict__ dq, int B, int H, int N,
-                                                          float scale) {
+                                                          float scale, int* status) {
   constexpr int TPR = D / 8;
   const int64_t rows = static_cast<int64_t>(B) * H * N;
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TPR;
@@ -168,6 +171,10 @@ __global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restric
   const int64_t bh = row / N;
   const int n = static_cast<int>(row % N);
   const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
+  if (!FA_IN_BOUNDS(row * D + part * 8 + 8 <= rows * D &&
+                        ((static_cast<int64_t>(b) * N + n) * H + h) * D + part * 8 + 8 <= rows * D,
+                    status, 221))
+    return;
   const float4* a = reinterpret_cast<const float4*>(dq_acc + row * D + part * 8);
   const float4 a0 = a[0], a1 = a[1];
   uint4 r;
@@ -291,8 +298,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&tm_dq);
       mbar_arrive_expect_tx(&sm.kv_full, 2 * Cfg::kTileBytes);
       for (int c = 0; c < Cfg::kChunks; ++c) {
-        tma_load_4d(sm.k + c * Cfg::kChunkBytes, &tm_k, &sm.kv_full, c * 64, hkv, j * 128, b);
-        tma_load_4d(sm.v + c * Cfg::kChunkBytes, &tm_v, &sm.kv_full, c * 64, hkv, j * 128, b);
+        if (FA_IN_BOUNDS(b < B && hkv < H_kv && j * 128 < N && c * 64 < D, status, 211)) {
+          tma_load_4d(sm.k + c * Cfg::kChunkBytes, &tm_k, &sm.kv_full, c * 64, hkv, j * 128, b);
+          tma_load_4d(sm.v + c * Cfg::kChunkBytes, &tm_v, &sm.kv_full, c * 64, hkv, j * 128, b);
+        }
       }
     }
     const int npad = nkb * 128;
@@ -312,9 +321,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // Q_i tile plus the block's LSE2 and D runs (512 bytes each, padded rows)
         mbar_arrive_expect_tx(&sm.q_full[st], Cfg::kTileBytes + 2 * 512);
         for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_4d(sm.q[st] + c * Cfg::kChunkBytes, &tm_q, &sm.q_full[st], c * 64, h, i * 128, b);
-        bulk_load(sm.lse2[st], lse2g + ridx, 512, &sm.q_full[st]);
-        bulk_load(sm.dd[st], dsum + ridx, 512, &sm.q_full[st]);
+          if (FA_IN_BOUNDS(h < H && i >= 0 && i * 128 < N && c * 64 < D, status, 212))
+            tma_load_4d(sm.q[st] + c * Cfg::kChunkBytes, &tm_q, &sm.q_full[st], c * 64, h, i * 128, b);
+        if (FA_IN_BOUNDS(ridx >= 0 && ridx + 128 <= static_cast<int64_t>(B) * H * npad, status, 213)) {
+          bulk_load(sm.lse2[st], lse2g + ridx, 512, &sm.q_full[st]);
+          bulk_load(sm.dd[st], dsum + ridx, 512, &sm.q_full[st]);
+        }
       }
       ++q_issued;
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.do_empty, (idx & 1) ^ 1, wc));
@@ -322,7 +334,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (lane == 0) {
         mbar_arrive_expect_tx(&sm.do_full, Cfg::kTileBytes);
         for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_4d(sm.dO + c * Cfg::kChunkBytes, &tm_do, &sm.do_full, c * 64, h, i * 128, b);
+          if (FA_IN_BOUNDS(h < H && i >= 0 && i * 128 < N && c * 64 < D, status, 212))
+            tma_load_4d(sm.dO + c * Cfg::kChunkBytes, &tm_do, &sm.do_full, c * 64, h, i * 128, b);
       }
       ++do_issued;
     }
@@ -522,7 +535,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t a[32];
         tmem_ld32(tAcc + c, a);
         tmem_wait_ld();
-        if (kg < N) {
+        if (kg < N && FA_IN_BOUNDS(kg >= 0 && ((static_cast<int64_t>(b) * N + kg) * H_kv + hkv) * D + c + 32 <=
+                                                   static_cast<int64_t>(B) * N * H_kv * D,
+                                   status, 214)) {
           uint4* pv = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
           for (int x = 0; x < 4; ++x)
@@ -580,7 +595,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int q0 = (i0 + idx % nper) * 128 + 32 * w;
         const int bh = b * H + hkv * group + idx / nper;  // query head: row block of the accumulator
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) tma_reduce_add_3d(&tm_dq, stg + c * 4096, 32 * c, q0, bh);
+        for (int c = 0; c < D / 32; ++c)
+          if (FA_IN_BOUNDS(bh < B * H && q0 >= 0 && q0 < nkb * 128, status, 215))
+            tma_reduce_add_3d(&tm_dq, stg + c * 4096, 32 * c, q0, bh);
         bulk_commit_group();
         bulk_wait_group_read0();
         mbar_arrive(&sm.stg_free[slot]);

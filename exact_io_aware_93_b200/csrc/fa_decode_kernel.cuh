@@ -108,6 +108,8 @@ struct DecArgs {
   int B, H, H_kv, N_q, N_kv, window, causal;
   int R;                   // row copies per tile (dec_copies of M)
   float scale_log2;
+  long long slots;         // partial slots in part_lse / part_o (for the checking build)
+  int* status;             // device status word (the merge kernel's bounds checks)
 };
 
 // Cached length of sequence b (clamped to the capacity), the first key tile any of its
@@ -282,8 +284,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         mbar_arrive_expect_tx(&sm.q_full[qi], static_cast<uint32_t>(R * Cfg::kChunks * 128 * M));
         for (int cp = 0; cp < R; ++cp)
           for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_4d(sm.q[qi] + c * Cfg::kChunkBytes + cp * kCopyRows * 128, &tm_q, &sm.q_full[qi], c * 64,
-                        s.kvh * G, 0, s.b);
+            if (FA_IN_BOUNDS(s.b < a.B && s.kvh * G + G <= a.H && c * 64 < D, status, 301))
+              tma_load_4d(sm.q[qi] + c * Cfg::kChunkBytes + cp * kCopyRows * 128, &tm_q, &sm.q_full[qi], c * 64,
+                          s.kvh * G, 0, s.b);
         ++qc;
         // K/V tiles in the order the MMA warp consumes them: K0, K1, then V_t, K_{t+2}
         auto load = [&](const CUtensorMap* m, int t) -> bool {
@@ -291,8 +294,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           if (!mbar_wait(&sm.kv_empty[slot], ((it / NS) & 1) ^ 1, wc)) return false;
           mbar_arrive_expect_tx(&sm.kv_full[slot], Cfg::kTileBytes);
           for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_4d(sm.kv[slot] + c * Cfg::kChunkBytes, m, &sm.kv_full[slot], c * 64, s.kvh, (s.kt0 + t) * 128,
-                        s.b);
+            if (FA_IN_BOUNDS(s.b < a.B && s.kvh < a.H_kv && s.kt0 + t >= 0 && (s.kt0 + t) * 128 < a.N_kv, status, 302))
+              tma_load_4d(sm.kv[slot] + c * Cfg::kChunkBytes, m, &sm.kv_full[slot], c * 64, s.kvh,
+                          (s.kt0 + t) * 128, s.b);
           ++it;
           return true;
         };
@@ -563,7 +567,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         for (int x = 0; x < 32; ++x)
           v[x] = (a0 * __uint_as_float(o0[x]) + (has1 ? a1 * __uint_as_float(o1[x]) : 0.f)) * inv;
         if (real) {
-          if (direct) {
+          if (direct && FA_IN_BOUNDS(((static_cast<int64_t>(b) * a.N_q + iq) * a.H + h) * D + c + 32 <=
+                                         static_cast<int64_t>(a.B) * a.N_q * a.H * D,
+                                     status, 303)) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<typename ElemOps<E>::T*>(a.out) +
                                                   ((static_cast<int64_t>(b) * a.N_q + iq) * a.H + h) * D + c);
 #pragma unroll
@@ -571,7 +577,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
               dst[x] = make_uint4(ElemOps<E>::pack(v[8 * x], v[8 * x + 1]), ElemOps<E>::pack(v[8 * x + 2], v[8 * x + 3]),
                                   ElemOps<E>::pack(v[8 * x + 4], v[8 * x + 5]),
                                   ElemOps<E>::pack(v[8 * x + 6], v[8 * x + 7]));
-          } else {
+          } else if (!direct && FA_IN_BOUNDS(slot >= 0 && slot < a.slots, status, 304)) {
             float4* dst = reinterpret_cast<float4*>(a.part_o + (slot * M + rc) * D + c);
 #pragma unroll
             for (int x = 0; x < 8; ++x) dst[x] = make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
@@ -580,8 +586,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
       if (real) {
         if (direct) {
-          a.lse[(static_cast<int64_t>(b) * a.H + h) * a.N_q + iq] = lse_l;
-        } else {
+          if (FA_IN_BOUNDS((static_cast<int64_t>(b) * a.H + h) * a.N_q + iq < static_cast<int64_t>(a.B) * a.H * a.N_q,
+                           status, 305))
+            a.lse[(static_cast<int64_t>(b) * a.H + h) * a.N_q + iq] = lse_l;
+        } else if (FA_IN_BOUNDS(slot >= 0 && slot < a.slots, status, 306)) {
           a.part_lse[(slot * M + rc) * 2 + 0] = lse_l;
           a.part_lse[(slot * M + rc) * 2 + 1] = lse_r;
         }
@@ -633,6 +641,7 @@ __global__ void __launch_bounds__(128) fa_decode_merge_kernel(const DecArgs a) {
   // partial results of this pair: slots (c + p) * R + copy for CTAs c in [cf, cl]
   const int s0 = (cf + p) * a.R;
   const int s1 = (cl + p) * a.R + a.R - 1;
+  if (!FA_IN_BOUNDS(s0 >= 0 && s1 < a.slots && 2 + b < 2 + a.B, a.status, 307)) return;
   for (int r = warp; r < M; r += 4) {
     float mx_l = -INFINITY, mx_r = -INFINITY;
     for (int c = s0 + lane; c <= s1; c += 32) {

@@ -283,8 +283,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (!ok) break;
           mbar_arrive_expect_tx(&sm.q_full[i], Cfg::kTileBytes);
           for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_4d(sm.q[i] + c * Cfg::kChunkBytes, &tm_q, &sm.q_full[i], c * Cfg::kChunkElems, ti.h,
-                        (ti.qb0 + i) * kBM, ti.b);
+            if (FA_IN_BOUNDS(ti.b < B && ti.h < H && (ti.qb0 + i) * kBM < N && c * Cfg::kChunkElems < D, status, 101))
+              tma_load_4d(sm.q[i] + c * Cfg::kChunkBytes, &tm_q, &sm.q_full[i], c * Cfg::kChunkElems, ti.h,
+                          (ti.qb0 + i) * kBM, ti.b);
           ++qcnt[i];
         }
         // K/V stream: the union of both blocks' ranges (block 1's range starts and ends later)
@@ -298,8 +299,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_arrive_expect_tx(&sm.kv_full[s], Cfg::kTileBytes);
             const CUtensorMap* m = kv ? &tm_v : &tm_k;
             for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_4d(sm.kv[s] + c * Cfg::kChunkBytes, m, &sm.kv_full[s], c * Cfg::kChunkElems, hkv, j * kBN,
-                          ti.b);
+              if (FA_IN_BOUNDS(ti.b < B && hkv < H_kv && j >= 0 && j * kBN < N && c * Cfg::kChunkElems < D, status,
+                               102))
+                tma_load_4d(sm.kv[s] + c * Cfg::kChunkBytes, m, &sm.kv_full[s], c * Cfg::kChunkElems, hkv,
+                            j * kBN, ti.b);
           }
         }
       }
@@ -533,13 +536,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int x = 0; x < 16; ++x)
           pk[x] = ElemOps<E == Elem::kE4M3 ? Elem::kBf16 : E>::pack(__uint_as_float(o[2 * x]) * inv_l,
                                                                    __uint_as_float(o[2 * x + 1]) * inv_l);
-        if (live) {
+        if (live && FA_IN_BOUNDS(((static_cast<int64_t>(ti.b) * N + row) * H + ti.h) * D + c + 32 <=
+                                     static_cast<int64_t>(B) * N * H * D && ti.h < H && row >= 0,
+                                 status, 103)) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
           for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
         }
       }
-      if (live) lse[(static_cast<int64_t>(ti.b) * H + ti.h) * N + row] = (m_ref + lg2_approx(l)) * kLn2;
+      if (live && FA_IN_BOUNDS((static_cast<int64_t>(ti.b) * H + ti.h) * N + row < static_cast<int64_t>(B) * H * N,
+                               status, 104))
+        lse[(static_cast<int64_t>(ti.b) * H + ti.h) * N + row] = (m_ref + lg2_approx(l)) * kLn2;
       tc_fence_before();
     }
   }

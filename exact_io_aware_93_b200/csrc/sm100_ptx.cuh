@@ -92,6 +92,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// ---------------------------------------------------------------- checking build
+// Compiled with -DFA_CHECKS, every TMA coordinate and every global index a kernel computes is
+// compared with the extent of the tensor it addresses before the access.  A violation records
+// FA_ERR_BOUNDS (8) and the check's site in the device status word, and the access is
+// skipped: a skipped TMA load leaves its barrier short of bytes, so the waiting role's bounded
+// wait runs out and the kernel unwinds.  Without FA_CHECKS the checks compile to nothing.
+#ifdef FA_CHECKS
+__device__ __noinline__ void bounds_fail(int* status, int site) {
+  atomicCAS(status, 0, 8 /* FA_ERR_BOUNDS */);
+  atomicCAS(status + 1, 0, site);
+}
+#define FA_IN_BOUNDS(cond, status, site) ((cond) ? true : (::fa::bounds_fail((status), (site)), false))
+#else
+#define FA_IN_BOUNDS(cond, status, site) true
+#endif
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

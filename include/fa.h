@@ -53,11 +53,24 @@ typedef enum {
   FA_ERR_DEVICE = 4,      /* no usable CUDA device, or the current device is not sm_100 */
   FA_ERR_LAUNCH = 5,      /* kernel attribute setup or launch failed */
   FA_ERR_TIMEOUT = 6,     /* a kernel abandoned a bounded wait (reported by fa_get_status) */
-  FA_ERR_WORKSPACE = 7    /* workspace pointer NULL or smaller than the required size */
+  FA_ERR_WORKSPACE = 7,   /* workspace pointer NULL or smaller than the required size */
+  FA_ERR_BOUNDS = 8       /* checking build only: a kernel's index left its tensor (fa_get_status) */
 } fa_status;
 
-/* Library ABI version (this header: 4). */
+/* Library ABI version (this header: 5). */
 int fa_abi_version(void);
+
+/*
+ * The checking build.  libfa_b200_checks.so is the same library compiled with FA_CHECKS:
+ * before every TMA copy and every global load or store it computes, each kernel compares the
+ * coordinates or index with the extent of the tensor addressed.  A violation records
+ * FA_ERR_BOUNDS and the check's site in the device status word and skips the access (a
+ * skipped copy leaves its barrier short, so the kernel unwinds through its bounded waits);
+ * fa_get_status() then returns FA_ERR_BOUNDS.  It stands in for a memory checker where none
+ * can run, and is slower; results are otherwise the same as the release library's.
+ * fa_checks_enabled() returns 1 in the checking build and 0 in the release build.
+ */
+int fa_checks_enabled(void);
 
 /*
  * Problem description for the _ex entry points.
@@ -277,9 +290,19 @@ fa_status fa_decode(const fa_decode_problem* problem, const void* q, const void*
 fa_status fa_selftest_wait_timeout(unsigned int timeout_us, void* stream);
 
 /*
+ * Checking-build self-test: launches one warp whose bounds check is given an index outside
+ * its (one-element, shared-memory) target, so the check fails by construction and the access
+ * is skipped; nothing outside the target is touched.  In the checking build the kernel
+ * records FA_ERR_BOUNDS and a following fa_get_status() returns it; the release build has no
+ * checks and returns FA_ERR_UNSUPPORTED without launching.  FA_ERR_DEVICE without an sm_100
+ * device, FA_ERR_LAUNCH if the launch fails, else FA_OK.
+ */
+fa_status fa_selftest_bounds(void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of the
- * current device: FA_OK, or FA_ERR_TIMEOUT if a kernel gave up a bounded wait
- * since the last call.  Returns FA_ERR_DEVICE if the stream or device reports a
+ * current device: FA_OK, FA_ERR_TIMEOUT if a kernel gave up a bounded wait since the
+ * last call, or (checking build) FA_ERR_BOUNDS if a bounds check failed.  Returns FA_ERR_DEVICE if the stream or device reports a
  * CUDA error.
  */
 fa_status fa_get_status(void* stream);

@@ -46,7 +46,8 @@ def test_status_strings(lib):
     assert lib.fa_status_string(0) == b"FA_OK"
     assert lib.fa_status_string(6) == b"FA_ERR_TIMEOUT"
     assert lib.fa_status_string(99) == b"FA_ERR_UNKNOWN"
-    assert lib.fa_abi_version() == 4
+    assert lib.fa_status_string(8) == b"FA_ERR_BOUNDS"
+    assert lib.fa_abi_version() == 5
 
 
 def _fwd(lib, q=0x10000, k=0x10000, v=0x10000, o=0x10000, lse=0x10000, B=1, H=1, N=16, d=64,
@@ -197,3 +198,19 @@ def test_e4m3_validation_codes(lib):
     import torch
     if not torch.cuda.is_available():
         assert call() == 4                    # valid, no sm_100 device here
+
+
+def test_checking_build_exports_the_same_symbols_and_says_so(lib):
+    chk = ctypes.CDLL(fabuild.CHECKS_LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(chk, name), f"{name} declared in include/*.h but not exported by the checking build"
+    assert lib.fa_checks_enabled() == 0
+    assert chk.fa_checks_enabled() == 1
+    # the release build has no checks: its self-test refuses before touching a device
+    lib.fa_selftest_bounds.argtypes = [ctypes.c_void_p]
+    assert lib.fa_selftest_bounds(None) == 2      # FA_ERR_UNSUPPORTED
+
+
+def test_checking_build_keeps_the_register_contract():
+    log = open(os.path.join(os.path.dirname(fabuild.CHECKS_LIB_PATH), "build_checks.log")).read()
+    fabuild.check_register_contract(log)
