@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd.restype = i
     L.fa_get_status.argtypes = [vp]
     L.fa_get_status.restype = i
+    L.fa_get_status_site.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    L.fa_get_status_site.restype = i
     L.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
     L.fa_selftest_wait_timeout.restype = i
     L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
@@ -308,6 +310,17 @@ def get_status(device: torch.device | None = None) -> int:
     with torch.cuda.device(dev):
         s = torch.cuda.current_stream(dev)
         return int(lib().fa_get_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def get_status_site(device: torch.device | None = None) -> tuple[int, int]:
+    """As get_status, and also where the first recorded error arose: the site number of the
+    wait that ran out or of the bounds check that failed (0 when none was recorded)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    site = ctypes.c_int(0)
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev)
+        st = int(lib().fa_get_status_site(ctypes.c_void_p(s.cuda_stream), ctypes.byref(site)))
+    return st, int(site.value)
 
 
 def selftest_wait_timeout(timeout_us: int = 20000) -> int:

@@ -589,7 +589,8 @@ fa_status fa_selftest_bounds(void* stream) {
 #endif
 }
 
-fa_status fa_get_status(void* stream) {
+fa_status fa_get_status_site(void* stream, int* site) {
+  if (site) *site = 0;
   DeviceInfo* di = nullptr;
   fa_status st = current_device(&di);
   if (st != FA_OK) return st;
@@ -604,7 +605,10 @@ fa_status fa_get_status(void* stream) {
     cudaGetLastError();
     return FA_ERR_DEVICE;
   }
+  if (site) *site = word[1];
   return word[0] == 0 ? FA_OK : static_cast<fa_status>(word[0]);
 }
+
+fa_status fa_get_status(void* stream) { return fa_get_status_site(stream, nullptr); }
 
 }  // extern "C"

@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp walks the issuer's path; one elected lane issues each MMA and commit
       const WaitCtx wc{&sm.abort_flag, status, 12};
       constexpr uint32_t kT = ElemOps<E>::kMmaType;
       constexpr uint32_t idesc_sdp = idesc_kind_f16(128, 128, 0, 0, kT);  // K-major x K-major
@@ -366,14 +366,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * Cfg::kChunkBytes + (kk % 4) * 32) >> 4;
-          umma_ss(tD, da + off, db + off, idesc_sdp, kk > 0);
+          umma_ss_w(tD, da + off, db + off, idesc_sdp, kk > 0);
         }
       };
-      bool ok = mbar_wait(&sm.kv_full, 0, wc) && mbar_wait(&sm.q_full[0], 0, wc);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.kv_full, 0, wc));
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.q_full[0], 0, wc));
       if (ok) {
         tc_fence_after();
         kmaj_gemm(tS, dk_kmaj, sdesc_sw128(smem_u32(sm.q[0]), 16, 1024));  // S^T for the first block
-        umma_commit(&sm.s_full);
+        umma_commit_w(&sm.s_full);
       }
       const uint64_t ddo_k = sdesc_sw128(smem_u32(sm.dO), 16, 1024);
       const uint64_t ddo_mn = sdesc_sw128(smem_u32(sm.dO), Cfg::kChunkBytes, 1024);
@@ -381,31 +382,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int st = idx & 1;
         const uint64_t dq_mn = sdesc_sw128(smem_u32(sm.q[st]), Cfg::kChunkBytes, 1024);
         if (idx > 0) {
-          ok = mbar_wait(&sm.dq_free, (idx - 1) & 1, wc);  // dQ_{i-1} copied out of the dP columns
+          // dQ_{i-1} copied out of the dP columns
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_free, (idx - 1) & 1, wc));
           if (!ok) break;
         }
-        ok = mbar_wait(&sm.do_full, idx & 1, wc);
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.do_full, idx & 1, wc));
         if (!ok) break;
         tc_fence_after();
         kmaj_gemm(tDP, dv_kmaj, ddo_k);  // dP^T = V dO^T
-        umma_commit(&sm.dp_full);
-        ok = mbar_wait(&sm.p_ready, idx & 1, wc);
+        umma_commit_w(&sm.dp_full);
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_ready, idx & 1, wc));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO   (K = 128 queries)
-          umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, ddo_mn + ((kk * 2048) >> 4), idesc_acc,
-                  (kk > 0) || (idx > 0));
+          umma_ts_w(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, ddo_mn + ((kk * 2048) >> 4), idesc_acc,
+                    (kk > 0) || (idx > 0));
         }
-        umma_commit(&sm.do_empty);  // dO_i is no longer read once dP and dV complete
+        umma_commit_w(&sm.do_empty);  // dO_i is no longer read once dP and dV complete
         if (idx + 1 < ni) {  // next block's S^T, into the columns P^T just left
-          ok = mbar_wait(&sm.q_full[st ^ 1], ((idx + 1) >> 1) & 1, wc);
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full[st ^ 1], ((idx + 1) >> 1) & 1, wc));
           if (!ok) break;
           tc_fence_after();
           kmaj_gemm(tS, dk_kmaj, sdesc_sw128(smem_u32(sm.q[st ^ 1]), 16, 1024));
-          umma_commit(&sm.s_full);
+          umma_commit_w(&sm.s_full);
         }
-        ok = mbar_wait(&sm.ds_ready, idx & 1, wc);
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.ds_ready, idx & 1, wc));
         if (!ok) break;
         tc_fence_after();
         // dK += dS^T Q (dS^T read K-major from shared memory) and dQ = dS K (K = 128 keys, into
@@ -413,14 +415,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4;
-          umma_ss(tDK, dds_k + off, dq_mn + ((kk * 2048) >> 4), idesc_acc, (kk > 0) || (idx > 0));
-          umma_ss(tDP, dds + ((kk * 2048) >> 4), dk_mn + ((kk * 2048) >> 4), idesc_dq, kk > 0);
+          umma_ss_w(tDK, dds_k + off, dq_mn + ((kk * 2048) >> 4), idesc_acc, (kk > 0) || (idx > 0));
+          umma_ss_w(tDP, dds + ((kk * 2048) >> 4), dk_mn + ((kk * 2048) >> 4), idesc_dq, kk > 0);
         }
-        umma_commit(&sm.q_empty[st]);
-        umma_commit(&sm.dq_full);
+        umma_commit_w(&sm.q_empty[st]);
+        umma_commit_w(&sm.dq_full);
       }
-      umma_commit(&sm.acc_done);
-      umma_commit(&sm.mma_drain);
+      umma_commit_w(&sm.acc_done);
+      umma_commit_w(&sm.mma_drain);
       mbar_wait_drain(&sm.mma_drain, 0, status);
     }
     __syncwarp();

@@ -311,10 +311,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
     }
   } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer (whole warp
-    // waits; lane 0 issues; the warp zeroes stale value rows)
+    // ------------------------------------------------------------ MMA issuer (the whole warp
+    // waits and zeroes stale value rows; one elected lane issues each MMA and commit)
     const WaitCtx wc{&sm.abort_flag, status, 22};
-    const bool leader = lane == 0;
     constexpr uint32_t idesc_s = idesc_kind_f16(kM, kBN, 0, 0, ElemOps<E>::kMmaType);  // Q, K K-major
     constexpr uint32_t idesc_o = idesc_kind_f16(kM, D, 0, 1, ElemOps<E>::kMmaType);    // P in TMEM, V MN-major
     const uint32_t kv_addr0 = smem_u32(sm.kv[0]);
@@ -329,7 +328,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = ((kk / 4) * Cfg::kChunkBytes + (kk % 4) * 32) >> 4;
-        umma_ss(tS, dq + off, dk + off, idesc_s, kk > 0);
+        umma_ss_w(tS, dq + off, dk + off, idesc_s, kk > 0);
       }
     };
     auto issue_pv = [&](int i, int slot, uint32_t acc) {
@@ -338,7 +337,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const uint64_t dv = dv0 + static_cast<uint64_t>((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk)
-        umma_ts(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_o, (kk > 0) || acc);
+        umma_ts_w(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_o, (kk > 0) || acc);
     };
     auto wait_all = [&](uint64_t* bar, uint32_t parity) { return __all_sync(kFull, mbar_wait(bar, parity, wc)); };
 
@@ -363,13 +362,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         ok = take();
         if (!ok) break;
         tc_fence_after();
-        if (leader) {
-          issue_s(t, qi, slot);
-          umma_commit(&sm.s_full[t]);
-          umma_commit(&sm.kv_empty[slot]);
-          if (t == s.n - 1) umma_commit(&sm.q_empty[qi]);
-        }
-        __syncwarp();
+        issue_s(t, qi, slot);
+        umma_commit_w(&sm.s_full[t]);
+        umma_commit_w(&sm.kv_empty[slot]);
+        if (t == s.n - 1) umma_commit_w(&sm.q_empty[qi]);
       }
       for (int t = 0; t < s.n && ok; ++t) {
         const int i = t & 1;
@@ -395,31 +391,23 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           __syncwarp();
         }
         tc_fence_after();
-        if (leader) {
-          issue_pv(i, slot, t >= 2);
-          umma_commit(&sm.kv_empty[slot]);
-          if (t + 2 >= s.n) umma_commit(&sm.o_done[i]);
-        }
-        __syncwarp();
+        issue_pv(i, slot, t >= 2);
+        umma_commit_w(&sm.kv_empty[slot]);
+        if (t + 2 >= s.n) umma_commit_w(&sm.o_done[i]);
         if (t + 2 < s.n) {
           ok = take();  // K_{t+2}
           if (!ok) break;
           tc_fence_after();
-          if (leader) {
-            issue_s(i, qi, slot);
-            umma_commit(&sm.s_full[i]);
-            umma_commit(&sm.kv_empty[slot]);
-            if (t + 2 == s.n - 1) umma_commit(&sm.q_empty[qi]);
-          }
-          __syncwarp();
+          issue_s(i, qi, slot);
+          umma_commit_w(&sm.s_full[i]);
+          umma_commit_w(&sm.kv_empty[slot]);
+          if (t + 2 == s.n - 1) umma_commit_w(&sm.q_empty[qi]);
         }
       }
     }
     // Wait for every MMA issued to finish before the columns are freed.
-    if (leader) {
-      umma_commit(&sm.mma_drain);
-      mbar_wait_drain(&sm.mma_drain, 0, status);
-    }
+    umma_commit_w(&sm.mma_drain);
+    mbar_wait_drain(&sm.mma_drain, 0, status);
     __syncwarp();
   } else if (warp < 4 && (warp % kWarpsPerCopy) * kQuarterRows < M) {
     // ------------------------------------------------------------ softmax, both streams

@@ -147,12 +147,14 @@ __device__ __forceinline__ KvRange fwd_range(int qb, int nkb, int window) {
 }
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int* status) {
-  // Used only while unwinding after an abort: ignores the abort flag, still bounded.
+  // The final wait for issued MMAs, and every wait while unwinding after an abort: ignores
+  // the abort flag, still bounded; a timeout here is reported at site 98.
   const uint32_t a = smem_u32(bar);
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_test(a, parity)) {
     if (globaltimer_ns() - t0 > FA_WAIT_TIMEOUT_NS) {
-      atomicCAS(status, 0, 6);
+      atomicCAS(status, 0, 6 /* FA_ERR_TIMEOUT */);
+      atomicCAS(status + 1, 0, 98);
       return false;
     }
   }
@@ -316,7 +318,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp walks the issuer's path; one elected lane issues each MMA and commit
       const WaitCtx wc{&sm.abort_flag, status, 2};
       constexpr uint32_t idesc_s = idesc_kind_f16(128, kBN, 0, 0, ElemOps<E>::kMmaType);  // Q, K K-major
       constexpr uint32_t idesc_o = idesc_kind_f16(128, D, 0, 1, ElemOps<E>::kMmaType);    // P in TMEM, V MN-major
@@ -337,9 +339,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int kk = 0; kk < Cfg::kSSteps; ++kk) {
           const uint32_t off = ((kk / 4) * Cfg::kChunkBytes + (kk % 4) * 32) >> 4;
           if constexpr (E == Elem::kE4M3)
-            umma_ss_f8(tS, dq[i] + off, dk + off, idesc_s, kk > 0);
+            umma_ss_f8_w(tS, dq[i] + off, dk + off, idesc_s, kk > 0);
           else
-            umma_ss(tS, dq[i] + off, dk + off, idesc_s, kk > 0);
+            umma_ss_w(tS, dq[i] + off, dk + off, idesc_s, kk > 0);
         }
       };
       auto issue_pv = [&](int i, int slot, uint32_t acc) {
@@ -349,9 +351,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < Cfg::kPVSteps; ++kk) {
           if constexpr (E == Elem::kE4M3)
-            umma_ts_f8(tO, tP + kk * 8, dv + ((kk * Cfg::kKeysPerStep * 128) >> 4), idesc_o, (kk > 0) || acc);
+            umma_ts_f8_w(tO, tP + kk * 8, dv + ((kk * Cfg::kKeysPerStep * 128) >> 4), idesc_o, (kk > 0) || acc);
           else
-            umma_ts(tO, tP + kk * 8, dv + ((kk * Cfg::kKeysPerStep * 128) >> 4), idesc_o, (kk > 0) || acc);
+            umma_ts_w(tO, tP + kk * 8, dv + ((kk * Cfg::kKeysPerStep * 128) >> 4), idesc_o, (kk > 0) || acc);
         }
       };
 
@@ -364,57 +366,57 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int jhi = rg[1].hi > rg[0].hi ? rg[1].hi : rg[0].hi;
         auto in = [&](int i, int j) { return j >= rg[i].lo && j < rg[i].hi; };
         for (int i = 0; i < 2 && ok; ++i)
-          if (rg[i].hi > rg[i].lo) ok = mbar_wait(&sm.q_full[i], qcnt[i] & 1, wc);
+          if (rg[i].hi > rg[i].lo) ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full[i], qcnt[i] & 1, wc));
         if (!ok) break;
         // prologue: S_i for the first key block
         const int sk0 = it % NS;
-        ok = mbar_wait(&sm.kv_full[sk0], (it / NS) & 1, wc);
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.kv_full[sk0], (it / NS) & 1, wc));
         if (!ok) break;
         ++it;
         tc_fence_after();
         for (int i = 0; i < 2; ++i) {
           if (!in(i, jlo)) continue;
           issue_s(i, sk0);
-          umma_commit(&sm.s_full[i]);
-          if (rg[i].hi == jlo + 1) umma_commit(&sm.q_empty[i]);
+          umma_commit_w(&sm.s_full[i]);
+          if (rg[i].hi == jlo + 1) umma_commit_w(&sm.q_empty[i]);
         }
-        umma_commit(&sm.kv_empty[sk0]);
+        umma_commit_w(&sm.kv_empty[sk0]);
         for (int j = jlo; j < jhi && ok; ++j) {
           const int sv = it % NS;
-          ok = mbar_wait(&sm.kv_full[sv], (it / NS) & 1, wc);
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.kv_full[sv], (it / NS) & 1, wc));
           if (!ok) break;
           ++it;
           int skn = -1;
           if (j + 1 < jhi) {
             skn = it % NS;
-            ok = mbar_wait(&sm.kv_full[skn], (it / NS) & 1, wc);
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.kv_full[skn], (it / NS) & 1, wc));
             if (!ok) break;
             ++it;
           }
           for (int i = 0; i < 2 && ok; ++i) {
             if (in(i, j)) {
-              ok = mbar_wait(&sm.p_full[i], pcnt[i] & 1, wc);
+              ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_full[i], pcnt[i] & 1, wc));
               if (!ok) break;
               ++pcnt[i];
               tc_fence_after();
               issue_pv(i, sv, j > rg[i].lo);
-              if (j + 1 == rg[i].hi) umma_commit(&sm.o_done[i]);
+              if (j + 1 == rg[i].hi) umma_commit_w(&sm.o_done[i]);
             }
             if (in(i, j + 1)) {
               issue_s(i, skn);
-              umma_commit(&sm.s_full[i]);
-              if (j + 2 == rg[i].hi) umma_commit(&sm.q_empty[i]);
+              umma_commit_w(&sm.s_full[i]);
+              if (j + 2 == rg[i].hi) umma_commit_w(&sm.q_empty[i]);
             }
           }
           if (!ok) break;
-          umma_commit(&sm.kv_empty[sv]);
-          if (skn >= 0) umma_commit(&sm.kv_empty[skn]);
+          umma_commit_w(&sm.kv_empty[sv]);
+          if (skn >= 0) umma_commit_w(&sm.kv_empty[skn]);
         }
         for (int i = 0; i < 2; ++i)
           if (rg[i].hi > rg[i].lo) ++qcnt[i];
       }
       // Wait for every MMA issued to finish before the columns are freed.
-      umma_commit(&sm.mma_drain);
+      umma_commit_w(&sm.mma_drain);
       mbar_wait_drain(&sm.mma_drain, 0, status);
     }
     __syncwarp();

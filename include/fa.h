@@ -307,6 +307,17 @@ fa_status fa_selftest_bounds(void* stream);
  */
 fa_status fa_get_status(void* stream);
 
+/*
+ * fa_get_status, and in *site (if not NULL) where the first recorded error arose: for
+ * FA_ERR_TIMEOUT the wait that ran out (forward: 1 loads, 2 MMA, 3 and 4 the softmax of the
+ * first and second query block; backward: 11 loads, 12 MMA, 13 key rows, 14 dQ drain;
+ * decode: 21 loads, 22 MMA, 23 softmax; 98 the final wait for issued MMAs or a wait while
+ * unwinding after an abort; 99 the self-test),
+ * for FA_ERR_BOUNDS the check that failed (three-digit sites, 999 the self-test); 0 when
+ * none was recorded.  The sources name each site beside its wait or check.
+ */
+fa_status fa_get_status_site(void* stream, int* site);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,6 +29,7 @@ def chk():
     L.fa_decode.argtypes = [ctypes.POINTER(api.FaDecodeProblem), vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     L.fa_bwd_noalloc.argtypes = [vp] * 9 + [ci, ci, ci, ci, cf, ci, vp]
     L.fa_get_status.argtypes = [vp]
+    L.fa_get_status_site.argtypes = [vp, ctypes.POINTER(ci)]
     L.fa_selftest_bounds.argtypes = [vp]
     assert L.fa_checks_enabled() == 1
     return L
@@ -47,6 +48,11 @@ def test_a_failing_check_is_reported(chk):
     assert chk.fa_selftest_bounds(_st()) == 0
     assert _status(chk) == 8          # FA_ERR_BOUNDS, read and cleared
     assert _status(chk) == 0
+    assert chk.fa_selftest_bounds(_st()) == 0
+    site = ci(0)
+    torch.cuda.synchronize()
+    assert chk.fa_get_status_site(_st(), ctypes.byref(site)) == 8
+    assert site.value == 999          # the self-test's own check site
 
 
 CASES = [  # B, H, H_kv, N, d, causal, window, dtype

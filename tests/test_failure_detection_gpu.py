@@ -27,6 +27,13 @@ def test_bounded_wait_times_out_and_reports():
     assert torch.isfinite(o.float()).all()
 
 
+def test_status_site_names_the_wait_that_ran_out():
+    assert api.get_status_site() == (0, 0)
+    assert api.selftest_wait_timeout(20000) == 0
+    assert api.get_status_site() == (6, 99)             # FA_ERR_TIMEOUT at the self-test's wait
+    assert api.get_status_site() == (0, 0)              # read and cleared, site included
+
+
 def test_selftest_rejects_bad_bound():
     assert api.selftest_wait_timeout(0) == 1
     assert api.selftest_wait_timeout(2_000_000) == 1
