@@ -336,8 +336,9 @@ __global__ void fa_wait_timeout_selftest_kernel(uint64_t timeout_ns, int* status
 // ---------------------------------------------------------------- bounds-check self-test
 // One warp checks an index against a one-element target; lane 0's index is one past the
 // end, so in the checking build its check fails, records FA_ERR_BOUNDS and skips the store.
-// The array has a spare second element, so no build ever writes outside it.
-__global__ void fa_bounds_selftest_kernel(int* status) {
+// The array has a spare second element, so no build ever writes outside it.  Only the
+// checking build launches it.
+[[maybe_unused]] __global__ void fa_bounds_selftest_kernel(int* status) {
   __shared__ int target[2];
   const int idx = threadIdx.x == 0 ? 1 : 0;
   if (FA_IN_BOUNDS(idx < 1, status, 999)) target[idx] = static_cast<int>(threadIdx.x);

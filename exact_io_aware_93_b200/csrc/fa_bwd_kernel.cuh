@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const typename ElemOps<
   if (live) {
     const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
     const int64_t off = ((static_cast<int64_t>(b) * N + n) * H + h) * D + part * 8;
-    const int64_t elems = static_cast<int64_t>(B) * N * H * D;
+    [[maybe_unused]] const int64_t elems = static_cast<int64_t>(B) * N * H * D;  // checking build only
     if (!FA_IN_BOUNDS(off >= 0 && off + 8 <= elems && (bh * N + n) * D + part * 8 + 8 <= elems, status, 201)) return;
     const uint4 ov = *reinterpret_cast<const uint4*>(o + off);
     const uint4 dv = *reinterpret_cast<const uint4*>(dout + off);

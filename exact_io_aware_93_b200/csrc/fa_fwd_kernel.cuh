@@ -59,6 +59,10 @@ constexpr uint32_t kFwdRegsSoftmax = 200;
 constexpr uint32_t kFwdRegsOther = 104;
 static_assert(2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsOther <= kFwdThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
+// Arrivals that release one P tile: e4m3 rows arrive once per warp (measured 4% faster),
+// 16-bit rows once per thread (per-warp arrivals measured 1-3% slower there).
+template <Elem E>
+constexpr int kPArrivals = E == Elem::kE4M3 ? 4 : 128;
 constexpr float kTau = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
@@ -239,7 +243,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.q_empty[i], 1);
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i], 128);
+      mbar_init(&sm.p_full[i], kPArrivals<E>);
       mbar_init(&sm.o_done[i], 1);
     }
     for (int s = 0; s < NS; ++s) {
@@ -516,7 +520,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&sm.p_full[g]);
+        if constexpr (kPArrivals<E> == 4) {
+          __syncwarp();
+          if ((r & 31) == 0) mbar_arrive(&sm.p_full[g]);
+        } else {
+          mbar_arrive(&sm.p_full[g]);
+        }
       }
       if (!ok) break;
       // epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2
