@@ -173,9 +173,16 @@ fa_status launch_bwd(DeviceInfo& di, const CUtensorMap& mq, const CUtensorMap& m
                                                               lse, dsum, lse2, dq_acc, B, H, N, di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   const int nkb = (N + 127) / 128;
+  // Heads interleaved per group of the grid order: as many (batch, key/value head) pairs as
+  // keep their Q, dO, fp32 dQ rows and K, V within about 80 MB of L2.
+  const long long head_bytes =
+      static_cast<long long>(N) * D * (static_cast<long long>(H / H_kv) * (2 + 2 + 4) + 2 + 2);
+  long long hpg = (80ll << 20) / (head_bytes > 0 ? head_bytes : 1);
+  const long long bhkv = static_cast<long long>(B) * H_kv;
+  hpg = hpg < 1 ? 1 : (hpg > bhkv ? bhkv : hpg);
   kern<<<B * H_kv * nkb, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, mdq, lse2, dsum, static_cast<T*>(dk),
                                                            static_cast<T*>(dv), B, H, H_kv, N, window, scale,
-                                                           di.status);
+                                                           static_cast<int>(hpg), di.status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   fa::fa_bwd_post_kernel<D, E><<<ew_blocks, 256, 0, stream>>>(dq_acc, static_cast<T*>(dq), B, H, N, scale,
                                                                di.status);

@@ -224,7 +224,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ lse2g,
                        const float* __restrict__ dsum, typename ElemOps<E>::T* __restrict__ dk,
                        typename ElemOps<E>::T* __restrict__ dv,
-                       int B, int H, int H_kv, int N, int window, float scale, int* status) {
+                       int B, int H, int H_kv, int N, int window, float scale, int heads_per_group,
+                       int* status) {
   using Cfg = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {  // the layout relies on a 1 KB aligned base
@@ -236,12 +237,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
   const int nkb = (N + 127) / 128;
   const int group = H / H_kv;  // query heads sharing this key/value head
-  // Head-major order: the CTAs resident at any time cover only a few heads, so their dQ
-  // accumulator rows and Q/dO tiles stay in L2.  Within a head, key blocks go heaviest
-  // first (with causal masking block j meets nkb - j query blocks), so the grid ends on
-  // the lightest blocks.
-  const int bhkv = blockIdx.x / nkb;
-  const int j = blockIdx.x % nkb;
+  // Order: (batch, key/value head) pairs in groups of heads_per_group; within a group, key
+  // blocks heaviest first (with causal masking block j meets nkb - j query blocks), the
+  // group's heads interleaved.  The CTAs resident at any time cover one or two groups, so
+  // their dQ accumulator rows and Q/dO tiles stay in L2, and the grid ends on the lightest
+  // blocks of the last group instead of starting the last head's heaviest block near the end.
+  const int BHkv = B * H_kv;
+  const int grp = blockIdx.x / (heads_per_group * nkb);
+  const int g0 = grp * heads_per_group;
+  const int gsz = BHkv - g0 < heads_per_group ? BHkv - g0 : heads_per_group;
+  const int rem = blockIdx.x - grp * heads_per_group * nkb;
+  const int bhkv = g0 + rem % gsz;
+  const int j = rem / gsz;
   const int b = bhkv / H_kv, hkv = bhkv % H_kv;
   // query blocks that see key block j: i >= j when causal, and with a window only those
   // whose first query is within `window` of the block's last key
