@@ -47,6 +47,19 @@ def test_bwd_workload_fwdbwd_causal():
     assert max(err.values()) <= GRAD_TOL, err
 
 
+@pytest.mark.parametrize("B,H,N", [(2, 3, 12000), (1, 7, 10000)])
+def test_bwd_grid_groups_with_a_ragged_last_group(B, H, N):
+    """The backward grid walks (batch, head) pairs in groups sized to L2 (here 4 + 2 and
+    5 + 2 heads): every head of every group, sampled rows, against the oracle."""
+    d = 128
+    inp = make_inputs(B, H, N, d, seed=8100 + N, with_do=True)
+    g = _run(inp, True)
+    sampled = [(b, h, sample_rows(N, 48, head_row_seed(8100 + N, b, h)).numpy())
+               for b in range(B) for h in range(H)]
+    err = grad_errors(inp, g, d ** -0.5, True, [], sampled)
+    assert max(err.values()) <= GRAD_TOL, err
+
+
 def test_bwd_nondefault_scale():
     inp = make_inputs(1, 2, 384, 128, seed=77, with_do=True)
     g = _run(inp, True, scale=0.21)
