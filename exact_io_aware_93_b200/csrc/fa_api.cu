@@ -394,7 +394,7 @@ fa_status noalloc_scratch(void** out) {
 
 extern "C" {
 
-int fa_abi_version(void) { return 5; }
+int fa_abi_version(void) { return 6; }
 
 int fa_checks_enabled(void) {
 #ifdef FA_CHECKS

@@ -57,7 +57,7 @@ typedef enum {
   FA_ERR_BOUNDS = 8       /* checking build only: a kernel's index left its tensor (fa_get_status) */
 } fa_status;
 
-/* Library ABI version (this header: 5). */
+/* Library ABI version (this header: 6; 6 added fa_get_status_site). */
 int fa_abi_version(void);
 
 /*

@@ -47,7 +47,7 @@ def test_status_strings(lib):
     assert lib.fa_status_string(6) == b"FA_ERR_TIMEOUT"
     assert lib.fa_status_string(99) == b"FA_ERR_UNKNOWN"
     assert lib.fa_status_string(8) == b"FA_ERR_BOUNDS"
-    assert lib.fa_abi_version() == 5
+    assert lib.fa_abi_version() == 6
 
 
 def _fwd(lib, q=0x10000, k=0x10000, v=0x10000, o=0x10000, lse=0x10000, B=1, H=1, N=16, d=64,
