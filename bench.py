@@ -184,12 +184,15 @@ def clock_stats(samples, window, slack_s: float = 0.05):
 
 def choose_peak(clk, burst: float, sustained: float):
     """The tensor peak a timed region is compared with, chosen from that region's own clock
-    samples: the sustained (power-capped) cuBLAS figure when any in-region sample shows
-    sw_power_cap, else the burst figure.  Returns (peak, kind, rule)."""
+    samples: the sustained (power-capped) cuBLAS figure when more than half of the in-region
+    samples show sw_power_cap, else the burst figure (the larger denominator: a region that
+    ran mostly uncapped is not excused by a capped sample or two).  Returns
+    (peak, kind, rule)."""
     n, capped = clk.get("samples", 0) or 0, clk.get("power_cap_samples", 0) or 0
-    if capped > 0:
-        return sustained, "sustained", f"sw_power_cap active in {capped} of {n} in-region clock samples"
-    return burst, "burst", f"sw_power_cap active in 0 of {n} in-region clock samples"
+    rule = f"sw_power_cap active in {capped} of {n} in-region clock samples"
+    if n > 0 and 2 * capped > n:
+        return sustained, "sustained", rule + " (a majority)"
+    return burst, "burst", rule + (" (not a majority)" if capped else "")
 
 
 def pipelined_e2e(sets, host_in, in_names, out_names, compute, nsteps):

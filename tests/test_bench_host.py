@@ -86,9 +86,14 @@ def test_peak_follows_the_regions_own_clock_samples():
     # no in-region sample saw the power cap: burst peak, and the rule says on how many samples
     peak, kind, rule = bench.choose_peak({"samples": 3, "power_cap_samples": 0}, burst, sus)
     assert (peak, kind) == (burst, "burst") and "0 of 3" in rule
-    # one capped sample is enough for the sustained peak
-    peak, kind, rule = bench.choose_peak({"samples": 4, "power_cap_samples": 1}, burst, sus)
-    assert (peak, kind) == (sus, "sustained") and "1 of 4" in rule
+    # a capped sample or two in a mostly uncapped region: still the burst peak
+    peak, kind, rule = bench.choose_peak({"samples": 5, "power_cap_samples": 1}, burst, sus)
+    assert (peak, kind) == (burst, "burst") and "1 of 5" in rule
+    peak, kind, _ = bench.choose_peak({"samples": 6, "power_cap_samples": 3}, burst, sus)
+    assert (peak, kind) == (burst, "burst")
+    # a capped majority: the sustained peak
+    peak, kind, rule = bench.choose_peak({"samples": 24, "power_cap_samples": 15}, burst, sus)
+    assert (peak, kind) == (sus, "sustained") and "15 of 24" in rule
     # no samples at all: the burst peak (the larger denominator, so the smaller fraction)
     peak, kind, _ = bench.choose_peak({"samples": 0, "power_cap_samples": 0}, burst, sus)
     assert peak == burst
