@@ -50,7 +50,10 @@ class FAError(RuntimeError):
 
 
 def library_path() -> str:
-    return _build.LIB_PATH
+    """The release library, or the checking build (every kernel bounds-checks its TMA
+    coordinates and global indices and reports FA_ERR_BOUNDS) when the environment sets
+    FA_B200_CHECKS=1 before the first call."""
+    return _build.CHECKS_LIB_PATH if os.environ.get("FA_B200_CHECKS") == "1" else _build.LIB_PATH
 
 
 def lib() -> ctypes.CDLL:

@@ -35,3 +35,11 @@ def test_scratch_checks():
         api.check_scratch("workspace", torch.empty(10, 10)[:, ::2], CPU)
     with pytest.raises(ValueError):
         api.check_scratch("workspace", torch.empty(10), torch.device("cuda", 0))
+
+
+def test_checking_build_selected_by_environment(monkeypatch):
+    from exact_io_aware_93_b200 import build as fabuild
+    monkeypatch.delenv("FA_B200_CHECKS", raising=False)
+    assert api.library_path() == fabuild.LIB_PATH
+    monkeypatch.setenv("FA_B200_CHECKS", "1")
+    assert api.library_path() == fabuild.CHECKS_LIB_PATH

@@ -1,6 +1,9 @@
 """Seeded random configurations through the forward, backward and decode entry points,
 against the fp64 oracle: batch, heads, grouping, lengths, head dimension, masking and
-element type drawn together, so that combinations no hand-written case names get checked."""
+element type drawn together, so that combinations no hand-written case names get checked.
+FA_FUZZ_DRAWS=n widens each draw to n seeds (default 24)."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -10,6 +13,7 @@ from exact_io_aware_93_b200.inputs import make_decode_inputs, make_inputs
 from tests.parity import GRAD_TOL, LSE_TOL, O_TOL, decode_errors, fwd_errors, fwd_errors_gqa, grad_errors_gqa
 
 pytestmark = pytest.mark.gpu
+_DRAWS = int(os.environ.get("FA_FUZZ_DRAWS", "0"))
 
 
 def _fwdbwd_case(seed):
@@ -24,7 +28,7 @@ def _fwdbwd_case(seed):
     return dict(B=int(rng.integers(1, 3)), H=H, H_kv=h_kv, N=N, d=d, causal=causal, window=window, dtype=dtype)
 
 
-@pytest.mark.parametrize("seed", range(24))
+@pytest.mark.parametrize("seed", range(_DRAWS or 24))
 def test_fuzz_fwd_bwd(seed):
     c = _fwdbwd_case(10_000 + seed)
     inp = make_inputs(c["B"], c["H"], c["N"], c["d"], seed=20_000 + seed, with_do=True, H_kv=c["H_kv"],
@@ -43,8 +47,11 @@ def test_fuzz_fwd_bwd(seed):
         # rounding reaches 1e-2; judged by the excess over half an ulp (tests/parity.py)
         eo, el = fwd_errors_gqa(inp, o, lse, c["d"] ** -0.5, c["causal"], c["window"])
     assert eo <= O_TOL and el <= LSE_TOL, (c, eo, el)
+    # gradients: the error in excess of the roundings the method performs by design (O in D,
+    # P, dS, the outputs; tests/parity.py), which dominate near-zero gradients of rows that
+    # see one or two keys
     err = grad_errors_gqa(inp, {"dq": dq.cpu(), "dk": dk.cpu(), "dv": dv.cpu()}, c["d"] ** -0.5, c["causal"],
-                          c["window"])
+                          c["window"], bounded=True)
     assert max(err.values()) <= GRAD_TOL, (c, err)
 
 
@@ -65,7 +72,7 @@ def _decode_case(seed):
                 causal=causal, window=window, dtype=dtype)
 
 
-@pytest.mark.parametrize("seed", range(24))
+@pytest.mark.parametrize("seed", range(_DRAWS or 24))
 def test_fuzz_decode(seed):
     c = _decode_case(30_000 + seed)
     inp = make_decode_inputs(c["B"], c["H"], c["H_kv"], c["N_q"], c["N_kv"], c["d"], seed=40_000 + seed,

@@ -65,3 +65,64 @@ def test_e4m3_quantisation_recipe():
     t = make_inputs_e4m3(1, 2, 40, 128, seed=3, H_kv=1)
     assert t["q"].shape == (1, 40, 2, 128) and t["k"].shape == (1, 40, 1, 128)
     assert all(isinstance(t[n + "_descale"], float) and t[n + "_descale"] > 0 for n in "qkv")
+
+
+def _rounded_backward(q, k, v, do, scale, causal, window, dtype, drop_d=False):
+    """fp64 backward with exactly the roundings grad_rounding_bounds covers: O and P rounded to
+    `dtype`, D from the rounded O, dS rounded to `dtype`.  drop_d plants a real mistake."""
+    import oracle
+    o, _, p = oracle.dense_fwd(q, k, v, scale, causal, window)
+
+    def rnd(x):
+        return torch.tensor(x).to(dtype).double().numpy()
+    pt, ot = rnd(p), rnd(o)
+    dp = do @ v.T
+    dd = 0.0 if drop_d else (do * ot).sum(1)[:, None]
+    ds = rnd(pt * (dp - dd))
+    return scale * ds @ k, scale * ds.T @ q, pt.T @ do
+
+
+def _small_problems():
+    from exact_io_aware_93_b200.inputs import make_inputs
+    rng = np.random.default_rng(5)
+    for trial in range(40):
+        n = int(rng.choice([1, 2, 3, 5, 17, 64, 130]))
+        d = int(rng.choice([64, 128]))
+        causal = bool(rng.integers(0, 2))
+        window = int(rng.choice([-1, 0, 1, 9])) if causal else -1
+        dtype = torch.float16 if trial % 3 == 0 else torch.bfloat16
+        inp = make_inputs(1, 1, n, d, seed=700 + trial, with_do=True, dtype=dtype)
+        head = [inp[x][0, :, 0, :].double().numpy() for x in ("q", "k", "v", "do")]
+        yield head, d ** -0.5, causal, window, dtype
+
+
+def test_grad_rounding_bound_contains_the_methods_roundings():
+    """The bound holds element by element for a backward that performs exactly those
+    roundings, on small problems including rows that see one or two keys."""
+    import oracle
+    from tests.parity import grad_rounding_bounds
+    for (q, k, v, do), scale, causal, window, dtype in _small_problems():
+        ref = oracle.bwd_rows(q, k, v, do, scale, causal, window=window)
+        ref = (ref[0], ref[2], ref[3])
+        got = _rounded_backward(q, k, v, do, scale, causal, window, dtype)
+        bounds = grad_rounding_bounds(q, k, v, do, scale, causal, window, dtype)
+        for g, r, bd in zip(got, ref, bounds):
+            assert (np.abs(g - r) <= bd * (1 + 1e-9) + 1e-15).all()
+
+
+def test_grad_rounding_bound_does_not_excuse_a_dropped_term():
+    """Leaving D out of dS is caught: its error exceeds the bound by more than the tolerance."""
+    import oracle
+    from tests.parity import GRAD_TOL, grad_rounding_bounds
+    caught = 0
+    total = 0
+    for (q, k, v, do), scale, causal, window, dtype in _small_problems():
+        if q.shape[0] < 17:
+            continue
+        total += 1
+        dq_ref = oracle.bwd_rows(q, k, v, do, scale, causal, window=window)[0]
+        dq_bad = _rounded_backward(q, k, v, do, scale, causal, window, dtype, drop_d=True)[0]
+        bq = grad_rounding_bounds(q, k, v, do, scale, causal, window, dtype)[0]
+        excess = np.maximum(np.abs(dq_bad - dq_ref) - bq, 0.0).max() / max(np.abs(dq_ref).max(), 1e-3)
+        caught += excess > GRAD_TOL
+    assert total > 0 and caught == total
